@@ -1,0 +1,273 @@
+// C ABI of libtq (include/tq.h): argument checks on the host, then kernel launches.
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "tq_internal.h"
+
+namespace tq {
+
+int sm_count(int device) {
+  static int cached[64] = {0};
+  if (device < 0 || device >= 64) return 148;
+  if (cached[device] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[device] = n;
+  }
+  return cached[device];
+}
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_size(int dtype) {
+  return dtype == TQ_F32 ? 4 : (dtype == TQ_BF16 || dtype == TQ_F16) ? 2 : 0;
+}
+
+tq_status check_rows(const void* x, int dtype, int64_t n_rows, int64_t ld) {
+  if (n_rows < 0) return TQ_EINVAL;
+  if (dtype != TQ_F32 && dtype != TQ_BF16) return TQ_EUNSUPPORTED;
+  if (ld < kD || (ld * elem_size(dtype)) % 16 != 0) return TQ_EINVAL;
+  if (n_rows > 0 && (x == nullptr || !aligned16(x))) return TQ_EINVAL;
+  return TQ_OK;
+}
+
+tq_status check_key_planes(const tq_quantizer* q, const tq_key_planes& p) {
+  if (!p.idx || !p.norms) return TQ_EINVAL;
+  if (!aligned16(p.idx) || (reinterpret_cast<uintptr_t>(p.norms) & 3u)) return TQ_EINVAL;
+  if (q->mode == TQ_MODE_PROD) {
+    if (!p.signs || !aligned16(p.signs)) return TQ_EINVAL;
+  }
+  return TQ_OK;
+}
+
+tq_status check_cache(const tq_quantizer* q, const tq_kv_cache* c) {
+  if (!c) return TQ_EINVAL;
+  if (c->batch <= 0 || c->n_kv_heads <= 0 || c->capacity <= 0 || c->capacity % 16) return TQ_EINVAL;
+  if (c->d != kD) return TQ_EUNSUPPORTED;
+  if (!c->len_dev || !c->len_host) return TQ_EINVAL;
+  if (check_key_planes(q, c->keys) != TQ_OK) return TQ_EINVAL;
+  if (!aligned16(c->keys.norms)) return TQ_EINVAL;
+  if (c->value_bits != 0) {
+    if (c->value_bits != 2 && c->value_bits != 4) return TQ_EUNSUPPORTED;
+    if (c->value_group != 32) return TQ_EUNSUPPORTED;
+    if (!c->values.q || !c->values.params || !aligned16(c->values.q) || !aligned16(c->values.params))
+      return TQ_EINVAL;
+  }
+  for (int b = 0; b < c->batch; ++b)
+    if (c->len_host[b] < 0 || c->len_host[b] > c->capacity) return TQ_EINVAL;
+  return TQ_OK;
+}
+
+}  // namespace
+}  // namespace tq
+
+using namespace tq;
+
+extern "C" {
+
+int tq_abi_version(void) { return TQ_ABI_VERSION; }
+
+const char* tq_status_string(tq_status s) {
+  switch (s) {
+    case TQ_OK: return "ok";
+    case TQ_EINVAL: return "invalid argument";
+    case TQ_EUNSUPPORTED: return "unsupported configuration";
+    case TQ_ECAPACITY: return "cache capacity exceeded";
+    case TQ_ENOMEM: return "out of memory";
+    case TQ_ECUDA: return "CUDA error";
+    case TQ_ETIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+tq_status tq_host_tables(int d, int bits, int mode, uint64_t seed, const int32_t* outliers,
+                         int n_outlier, double* centroids, double* thresholds, int8_t* signs,
+                         int32_t* channels, uint16_t* s_rot_fp16) {
+  HostTables* t = new (std::nothrow) HostTables;
+  if (!t) return TQ_ENOMEM;
+  tq_key_layout_t lay;
+  const tq_status st = build_host_tables(d, bits, mode, seed, outliers, n_outlier, t, &lay);
+  if (st == TQ_OK) {
+    if (centroids) std::memcpy(centroids, t->cent, sizeof(t->cent));
+    if (thresholds) std::memcpy(thresholds, t->thr, sizeof(t->thr));
+    if (signs) std::memcpy(signs, t->signs, sizeof(t->signs));
+    if (channels) std::memcpy(channels, t->chan, sizeof(t->chan));
+    if (s_rot_fp16 && mode == TQ_MODE_PROD) std::memcpy(s_rot_fp16, t->s_rot, sizeof(t->s_rot));
+  }
+  delete t;
+  return st;
+}
+
+tq_status tq_build_codebook(int d, int bits, int mode, uint64_t seed,
+                            const int32_t* outlier_channels, int n_outlier, tq_quantizer** out) {
+  if (!out) return TQ_EINVAL;
+  *out = nullptr;
+  tq_quantizer* q = new (std::nothrow) tq_quantizer;
+  if (!q) return TQ_ENOMEM;
+  std::memset(q, 0, sizeof(*q));
+  tq_status st = build_host_tables(d, bits, mode, seed, outlier_channels, n_outlier, &q->host,
+                                   &q->layout);
+  if (st != TQ_OK) {
+    delete q;
+    return st;
+  }
+  q->d = d;
+  q->bits = bits;
+  q->mode = mode;
+  q->seed = seed;
+
+  DevTables* h = new (std::nothrow) DevTables;
+  if (!h) {
+    delete q;
+    return TQ_ENOMEM;
+  }
+  std::memset(h, 0, sizeof(*h));
+  const int nl0 = mode == TQ_MODE_MSE ? (1 << bits) : mode == TQ_MODE_PROD ? (1 << (bits - 1)) : (1 << (bits + 1));
+  for (int k = 0; k < nl0; ++k) h->cent[0][k] = static_cast<float>(q->host.cent[0][k]);
+  for (int k = 0; k + 1 < nl0; ++k) h->thr[0][k] = static_cast<float>(q->host.thr[0][k]);
+  if (mode == TQ_MODE_GROUPED) {
+    const int nl1 = 1 << bits;
+    for (int k = 0; k < nl1; ++k) h->cent[1][k] = static_cast<float>(q->host.cent[1][k]);
+    for (int k = 0; k + 1 < nl1; ++k) h->thr[1][k] = static_cast<float>(q->host.thr[1][k]);
+  }
+  for (int j = 0; j < kD; ++j) {
+    if (q->host.signs[j] < 0) h->sign_bits[j >> 5] |= 1u << (j & 31);
+    h->chan[j] = static_cast<uint8_t>(q->host.chan[j]);
+  }
+  if (mode == TQ_MODE_PROD) {
+    for (int r = 0; r < kD; ++r)
+      for (int c = 0; c < kD; ++c) {
+        const uint16_t v = q->host.s_rot[r * kD + c];
+        std::memcpy(&h->s_rot[r * kD + c], &v, 2);
+        std::memcpy(&h->s_rot_t[c * kD + r], &v, 2);
+      }
+  }
+  if (cudaGetDevice(&q->device) != cudaSuccess) {
+    delete h;
+    delete q;
+    return TQ_ECUDA;
+  }
+  if (cudaMalloc(&q->dev, sizeof(DevTables)) != cudaSuccess) {
+    delete h;
+    delete q;
+    return TQ_ENOMEM;
+  }
+  st = cudaMemcpy(q->dev, h, sizeof(DevTables), cudaMemcpyHostToDevice) == cudaSuccess ? TQ_OK : TQ_ECUDA;
+  delete h;
+  if (st != TQ_OK) {
+    cudaFree(q->dev);
+    delete q;
+    return st;
+  }
+  *out = q;
+  return TQ_OK;
+}
+
+void tq_free(tq_quantizer* q) {
+  if (!q) return;
+  if (q->dev) cudaFree(q->dev);
+  delete q;
+}
+
+tq_status tq_key_layout(const tq_quantizer* q, tq_key_layout_t* out) {
+  if (!q || !out) return TQ_EINVAL;
+  *out = q->layout;
+  return TQ_OK;
+}
+
+tq_status tq_quantize_keys(const tq_quantizer* q, const void* x, int dtype, int64_t n_rows,
+                           int64_t ld, tq_key_planes out, void* stream) {
+  if (!q) return TQ_EINVAL;
+  tq_status st = check_rows(x, dtype, n_rows, ld);
+  if (st != TQ_OK) return st;
+  if (n_rows == 0) return TQ_OK;
+  if ((st = check_key_planes(q, out)) != TQ_OK) return st;
+  if (q->mode != TQ_MODE_GROUPED && (reinterpret_cast<uintptr_t>(out.norms) & 3u)) return TQ_EINVAL;
+  return launch_quantize_keys(q, x, dtype, n_rows, ld, out, RowMap{nullptr, 0, 0, 0},
+                              static_cast<cudaStream_t>(stream));
+}
+
+tq_status tq_quantize_values(const void* v, int dtype, int64_t n_rows, int64_t ld, int d, int bits,
+                             int group, tq_value_planes out, void* stream) {
+  if (d != kD) return TQ_EUNSUPPORTED;
+  if (bits != 2 && bits != 4) return TQ_EUNSUPPORTED;
+  if (group != 32) return TQ_EUNSUPPORTED;
+  tq_status st = check_rows(v, dtype, n_rows, ld);
+  if (st != TQ_OK) return st;
+  if (n_rows == 0) return TQ_OK;
+  if (!out.q || !out.params || (reinterpret_cast<uintptr_t>(out.params) & 3u) ||
+      (reinterpret_cast<uintptr_t>(out.q) & 3u))
+    return TQ_EINVAL;
+  return launch_quantize_values(v, dtype, n_rows, ld, bits, out, RowMap{nullptr, 0, 0, 0},
+                                static_cast<cudaStream_t>(stream));
+}
+
+tq_status tq_append(const tq_quantizer* q, tq_kv_cache* c, const void* k_new, const void* v_new,
+                    int dtype, int n_tokens, void* stream) {
+  if (!q) return TQ_EINVAL;
+  tq_status st = check_cache(q, c);
+  if (st != TQ_OK) return st;
+  if (n_tokens < 0) return TQ_EINVAL;
+  if (n_tokens == 0) return TQ_OK;
+  if (dtype != TQ_F32 && dtype != TQ_BF16) return TQ_EUNSUPPORTED;
+  if (!k_new || !aligned16(k_new)) return TQ_EINVAL;
+  if (c->value_bits != 0 && (!v_new || !aligned16(v_new))) return TQ_EINVAL;
+  if (c->value_bits == 0 && v_new) return TQ_EINVAL;
+  for (int b = 0; b < c->batch; ++b)
+    if (static_cast<int64_t>(c->len_host[b]) + n_tokens > c->capacity) return TQ_ECAPACITY;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t rows = static_cast<int64_t>(c->batch) * c->n_kv_heads * n_tokens;
+  const RowMap map{c->len_dev, c->n_kv_heads, n_tokens, c->capacity};
+  if ((st = launch_quantize_keys(q, k_new, dtype, rows, kD, c->keys, map, s)) != TQ_OK) return st;
+  if (c->value_bits != 0) {
+    if ((st = launch_quantize_values(v_new, dtype, rows, kD, c->value_bits, c->values, map, s)) != TQ_OK)
+      return st;
+  }
+  if ((st = launch_advance_len(c->len_dev, c->batch, n_tokens, s)) != TQ_OK) return st;
+  for (int b = 0; b < c->batch; ++b) c->len_host[b] += n_tokens;
+  return TQ_OK;
+}
+
+tq_status tq_decode_workspace_bytes(const tq_kv_cache* c, int n_q_heads, size_t* bytes) {
+  if (!c || !bytes || n_q_heads <= 0 || c->batch <= 0 || c->capacity <= 0) return TQ_EINVAL;
+  *bytes = decode_workspace_bytes(c->batch, n_q_heads, c->capacity);
+  return TQ_OK;
+}
+
+tq_status tq_decode_attention(const tq_quantizer* q, const tq_kv_cache* c, const void* qv,
+                              int q_dtype, int n_q_heads, const int32_t* head_map, float sm_scale,
+                              void* out, int out_dtype, float* scores, int64_t scores_ld,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q) return TQ_EINVAL;
+  if (q->mode != TQ_MODE_PROD) return TQ_EUNSUPPORTED;
+  tq_status st = check_cache(q, c);
+  if (st != TQ_OK) return st;
+  if (n_q_heads <= 0 || n_q_heads > 512) return TQ_EINVAL;
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_EUNSUPPORTED;
+  if (!qv || !aligned16(qv)) return TQ_EINVAL;
+  if (head_map) {
+    for (int h = 0; h < n_q_heads; ++h)
+      if (head_map[h] < 0 || head_map[h] >= c->n_kv_heads) return TQ_EINVAL;
+  } else if (n_q_heads % c->n_kv_heads != 0) {
+    return TQ_EINVAL;
+  }
+  if (c->value_bits != 0) {
+    if (!out || !aligned16(out)) return TQ_EINVAL;
+    if (out_dtype != TQ_F32 && out_dtype != TQ_BF16) return TQ_EUNSUPPORTED;
+  } else if (out) {
+    return TQ_EINVAL;
+  }
+  int max_len = 0;
+  for (int b = 0; b < c->batch; ++b) max_len = c->len_host[b] > max_len ? c->len_host[b] : max_len;
+  if (scores && scores_ld < max_len) return TQ_EINVAL;
+  if (!workspace || !aligned16(workspace)) return TQ_EINVAL;
+  if (workspace_bytes < decode_workspace_bytes(c->batch, n_q_heads, c->capacity)) return TQ_EINVAL;
+  return launch_decode(q, c, qv, q_dtype, n_q_heads, head_map, sm_scale, out, out_dtype, scores,
+                       scores_ld, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,90 @@
+// Internal declarations of libtq: the device copy of a quantizer's tables, the host
+// quantizer object and the kernel launchers. Not part of the public ABI (include/tq.h).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/tq.h"
+
+namespace tq {
+
+constexpr int kD = 128;          // head dimension of the GPU path
+constexpr int kMaxLevels = 16;   // 4-bit codebook
+
+// Tables a kernel needs, in one device allocation per quantizer.
+// Row 0 of thr/cent is the full-width quantizer (grouped: the outlier group), row 1 the
+// grouped normal group. Thresholds and centroids are N(0,1)-scale: the kernels compare the
+// unnormalised Hadamard transform y = H (s . x) of a d_g-channel group against
+// t_k * ||x_g|| * sqrt(32 / d_g) (sqrt factor only for the 96-channel group), which is
+// the decision u_j = (Pi x)_j / ||x|| > t_k / sqrt(d_g).
+struct DevTables {
+  float thr[2][kMaxLevels];
+  float cent[2][kMaxLevels];
+  uint32_t sign_bits[4];   // bit j set <=> rotation sign s_j = -1 (grouped: 32 outlier, 96 normal)
+  uint8_t chan[kD];        // grouped: outlier channels ascending, then normal channels ascending
+  __half s_rot[kD * kD];   // prod: S_rot row-major (fp16-exact Gaussian)
+  __half s_rot_t[kD * kD]; // prod: S_rot transposed (column j of S_rot contiguous)
+};
+
+struct HostTables {
+  double cent[2][kMaxLevels];
+  double thr[2][kMaxLevels];
+  int8_t signs[kD];
+  int32_t chan[kD];
+  uint16_t s_rot[kD * kD];  // fp16 bits
+};
+
+// Host set-up (tq_host.cpp).
+tq_status build_host_tables(int d, int bits, int mode, uint64_t seed, const int32_t* outliers,
+                            int n_outlier, HostTables* t, tq_key_layout_t* layout);
+uint16_t float_to_half_bits_rn(double x);
+
+}  // namespace tq
+
+struct tq_quantizer {
+  int d, bits, mode;
+  uint64_t seed;
+  tq_key_layout_t layout;
+  tq::HostTables host;
+  tq::DevTables* dev;   // device copy
+  int device;           // CUDA device the copy lives on
+};
+
+namespace tq {
+
+// ---------------------------------------------------------------- kernel launchers
+
+// Where quantized rows are written. Contiguous: output row = input row. Cache: input row r
+// = ((b * n_kv_heads + h) * n_tokens + t) goes to cache row (b * n_kv_heads + h) * capacity
+// + len[b] + t, with len read on the device.
+struct RowMap {
+  const int32_t* len;   // nullptr => contiguous
+  int32_t n_kv_heads, n_tokens, capacity;
+};
+
+tq_status launch_quantize_keys(const tq_quantizer* q, const void* x, int dtype, int64_t n_rows,
+                               int64_t ld, tq_key_planes out, RowMap map, cudaStream_t st);
+tq_status launch_quantize_values(const void* v, int dtype, int64_t n_rows, int64_t ld, int bits,
+                                 tq_value_planes out, RowMap map, cudaStream_t st);
+tq_status launch_advance_len(int32_t* len, int batch, int n, cudaStream_t st);
+
+struct DecodePlan {
+  int n_groups;          // CTA head groups over all KV heads
+  int n_splits;          // context splits per (sequence, head group)
+  int tokens_per_split;  // multiple of 32
+  int max_len;
+};
+
+size_t decode_workspace_bytes(int batch, int n_q_heads, int capacity);
+tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* cache, const void* qv,
+                        int q_dtype, int n_q_heads, const int32_t* head_map, float sm_scale,
+                        void* out, int out_dtype, float* scores, int64_t scores_ld,
+                        void* workspace, size_t workspace_bytes, cudaStream_t st);
+
+int sm_count(int device);
+
+}  // namespace tq

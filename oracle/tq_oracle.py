@@ -379,16 +379,10 @@ def quantize_keys(q: Quantizer, X) -> dict:
         norms = [n16]
         out["n_exact"] = [np.sqrt(np.sum(X * X, axis=1))]
         if q.mode == "prod":
-            # [tutorial] algorithm overview: residual = k - decompress(...); QJL = sign(S @ r)
-            R = X - x_hat
-            rn = np.sqrt(np.sum(R * R, axis=1))
-            r16 = fp16_rn(fp32(rn))
-            SR = R @ q.S.T
-            sigma = (fp32(SR) >= 0).astype(np.int64)         # sign(0) counts as +1
+            sigma, margin_s, r16, rn = prod_residual_signs(q, X, idx, n16)
             out["sigma"] = sigma
             out["signs"] = pack_bits(sigma, 1)
-            with np.errstate(divide="ignore", invalid="ignore"):
-                out["sign_margin"] = np.where(rn[:, None] > 0, np.abs(SR) / rn[:, None], np.inf)
+            out["sign_margin"] = margin_s
             norms.append(r16)
             out["n_exact"].append(rn)
         out["norms"] = fp16_bits(np.stack(norms, axis=1))
@@ -410,6 +404,24 @@ def quantize_keys(q: Quantizer, X) -> dict:
     out["n_exact"] = exact
     assert out["idx"].shape == (n_rows, key_layout(q)["idx_bytes"])
     return out
+
+
+def prod_residual_signs(q: Quantizer, X: np.ndarray, idx: np.ndarray, n16: np.ndarray):
+    """QJL part of TurboQuantProd for given MSE codes and stored norms ([tutorial] algorithm
+    overview: residual = k - decompress(codes); sign(S @ residual)).
+
+    r = x - n16 Pi^T c[idx]; r16 = fp16(fp32(||r||)); sigma_j = [fp32((S r)_j) >= 0]
+    (sign(0) counts as +1). Returns (sigma, |S r| / ||r||, r16, ||r||)."""
+    X = np.asarray(X, dtype=np.float64)
+    x_hat = np.asarray(n16, dtype=np.float64)[:, None] * (q.cent[idx] @ q.Pi)
+    R = X - x_hat
+    rn = np.sqrt(np.sum(R * R, axis=1))
+    r16 = fp16_rn(fp32(rn))
+    SR = R @ q.S.T
+    sigma = (fp32(SR) >= 0).astype(np.int64)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        margin = np.where(rn[:, None] > 0, np.abs(SR) / rn[:, None], np.inf)
+    return sigma, margin, r16, rn
 
 
 def reconstruct_keys(q: Quantizer, planes: dict) -> np.ndarray:

@@ -1,0 +1,204 @@
+"""GPU parity of fused decode attention (tq_decode_attention) against the oracle.
+
+The packed caches are produced by the oracle's quantizer (never by the CUDA path) and
+uploaded, so these tests isolate the decode kernel; key-quantize parity is tested apart."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+from gpu_util import oracle_cache, require_cuda, to_device, to_np_planes, upload_cache
+from parity import check_attention, check_key_parity, check_scores
+
+pytestmark = pytest.mark.gpu
+
+import kv_cache_vector_fwht_b200 as tq  # noqa: E402
+
+
+def run_decode(qg, cache, Q, q_dtype, out_dtype, head_map=None, sm_scale=0.0, scores_ld=0):
+    dev = cache.len_dev.device
+    B, Hq, d = Q.shape
+    qt = to_device(Q, q_dtype)
+    out = torch.full((B, Hq, d), float("nan"), device=dev, dtype=out_dtype) if cache.value_bits else None
+    scores = torch.full((B, Hq, scores_ld), float("nan"), device=dev) if scores_ld else None
+    ws = tq.alloc_decode_workspace(cache, Hq)
+    tq.tq_decode_attention(qg, cache, qt, out, ws, head_map=head_map, sm_scale=sm_scale,
+                           scores=scores)
+    torch.cuda.synchronize()
+    return (out.float().cpu().numpy() if out is not None else None,
+            scores.cpu().numpy() if scores is not None else None, ws)
+
+
+def small_case(seed, B, Hq, Hkv, lengths, cap, bits, vbits):
+    g = W.rng(seed)
+    N = max(lengths)
+    K = W.round_bf16(W.scaled_gaussian_rows(g, B * Hkv * N).reshape(B, Hkv, N, 128))
+    V = W.round_bf16(W.gaussian(g, (B, Hkv, N, 128)))
+    Q = W.round_bf16(W.gaussian(g, (B, Hq, 128)))
+    qo = O.build_quantizer(128, bits, "prod", seed)
+    qg = tq.tq_build_codebook(128, bits, "prod", seed)
+    oc = oracle_cache(qo, K, V if vbits else None, vbits, lengths)
+    cache = tq.KVCache(qg, B, Hkv, cap, value_bits=vbits, device="cuda:0")
+    upload_cache(cache, oc)
+    return qo, qg, oc, cache, Q
+
+
+@pytest.mark.parametrize("bits,vbits", [(2, 2), (3, 2), (3, 4), (4, 4), (4, 2), (2, 4)])
+@pytest.mark.parametrize("q_dtype,out_dtype", [(torch.bfloat16, torch.float32),
+                                               (torch.float32, torch.bfloat16)])
+def test_decode_small_ragged(bits, vbits, q_dtype, out_dtype):
+    """Several context splits, a ragged tail and sequences of different lengths."""
+    require_cuda()
+    qo, qg, oc, cache, Q = small_case(40 + bits + vbits, 2, 6, 2, [1000, 777], 1024, bits, vbits)
+    if q_dtype == torch.float32:
+        Q = W.gaussian(W.rng(5), Q.shape)
+    out, _, _ = run_decode(qg, cache, Q, q_dtype, out_dtype)
+    ref, _ = O.decode_attention(qo, oc, Q.astype(np.float64), value_bits=vbits)
+    err = check_attention(out, ref, out_dtype == torch.bfloat16)
+    print(bits, vbits, err)
+
+
+def test_decode_head_map_scale_and_scores():
+    require_cuda()
+    qo, qg, oc, cache, Q = small_case(7, 1, 5, 3, [600], 608, 3, 2)
+    hm = np.array([2, 0, 2, 1, 2])
+    out, sc, _ = run_decode(qg, cache, Q, torch.bfloat16, torch.float32, head_map=hm,
+                            sm_scale=0.05, scores_ld=608)
+    ref, rs = O.decode_attention(qo, oc, Q.astype(np.float64), head_map=hm, sm_scale=0.05,
+                                 value_bits=2, want_scores=True)
+    check_attention(out, ref, False)
+    n16 = O.fp16_from_bits(oc["k_norms"][0, :, :600, 0])
+    for h in range(5):
+        check_scores(sc[0, h, :600], rs[0][h], np.linalg.norm(Q[0, h]), n16[hm[h]])
+    assert np.all(np.isnan(sc[0, :, 600:]))      # nothing written beyond len
+
+
+def test_decode_empty_and_single_token_sequences():
+    require_cuda()
+    qo, qg, oc, cache, Q = small_case(8, 3, 4, 2, [0, 1, 300], 304, 3, 2)
+    out, _, ws = run_decode(qg, cache, Q, torch.bfloat16, torch.float32)
+    ref, _ = O.decode_attention(qo, oc, Q.astype(np.float64), value_bits=2)
+    assert np.all(out[0] == 0.0)                 # len 0 -> zeros
+    check_attention(out, ref, False)
+    vh = O.dequantize_values(oc["v_q"][1, 0, :1], oc["v_params"][1, 0, :1], 2, 128)[0]
+    assert np.allclose(out[1, 0], vh, atol=1e-6)  # one key -> its value
+    # the workspace is left reusable: a second call gives the same result
+    out2, _, _ = run_decode(qg, cache, Q, torch.bfloat16, torch.float32)
+    assert np.array_equal(out, out2)
+
+
+def test_score_workload():
+    """Score workload: 4096 fp32 keys (3-bit prod, seed 0), 8 fp32 queries as 8 query heads
+    on one KV head, key-only cache; outputs the 4096 x 8 estimate matrix. Also checks the
+    keys the GPU quantized against the oracle (end to end)."""
+    dev = require_cuda()
+    keys, queries = W.score_inputs()
+    qo = O.build_quantizer(128, 3, "prod", 0)
+    qg = tq.tq_build_codebook(128, 3, "prod", 0)
+    oc = oracle_cache(qo, keys[None, None], None, 0, [4096])
+    cache = tq.KVCache(qg, 1, 1, 4096, value_bits=0, device=dev)
+    upload_cache(cache, oc)
+    _, sc, _ = run_decode(qg, cache, queries[None], torch.float32, None, scores_ld=4096)
+    _, rs = O.decode_attention(qo, oc, queries[None].astype(np.float64), want_scores=True)
+    n16 = O.fp16_from_bits(oc["k_norms"][0, 0, :, 0])
+    worst = max(check_scores(sc[0, h], rs[0][h], np.linalg.norm(queries[h]), n16)
+                for h in range(8))
+    print("score rel err", worst)
+    # end to end: GPU-quantized keys scored on the GPU
+    cache2 = tq.KVCache(qg, 1, 1, 4096, value_bits=0, device=dev)
+    tq.tq_append(qg, cache2, to_device(keys[None, None], torch.float32))
+    gp = to_np_planes(cache2.key_planes())
+    check_key_parity(qo, keys.astype(np.float64), gp)
+    _, sc2, _ = run_decode(qg, cache2, queries[None], torch.float32, None, scores_ld=4096)
+    same = np.all(gp["idx"] == oc["k_idx"][0, 0], axis=1) & np.all(gp["signs"] == oc["k_signs"][0, 0], axis=1)
+    for h in range(8):
+        check_scores(sc2[0, h][same], rs[0][h][same], np.linalg.norm(queries[h]), n16[same])
+
+
+def _full_decode(cfg_id, sample_pairs, out_dtype):
+    require_cuda()
+    cfg = W.WORKLOADS[cfg_id]
+    B, Hq, Hkv, N = cfg["batch"], cfg["n_q_heads"], cfg["n_kv_heads"], cfg["ctx"]
+    K, V, Q, _ = W.decode_inputs(cfg_id, B, Hq, Hkv, N, planted=cfg.get("planted", 0))
+    qo = O.build_quantizer(128, cfg["key_bits"], "prod", cfg["qseed"])
+    qg = tq.tq_build_codebook(128, cfg["key_bits"], "prod", cfg["qseed"])
+    G = Hq // Hkv
+    vb = cfg["value_bits"]
+    # the oracle quantizes only the (b, kv) pairs that are checked; the rest of the cache
+    # holds the same data quantized on the GPU, which only feeds outputs not compared here
+    cap = N + 256
+    cache = tq.KVCache(qg, B, Hkv, cap, value_bits=vb, device="cuda:0")
+    tq.tq_append(qg, cache, to_device(K, torch.bfloat16), to_device(V, torch.bfloat16))
+    for b, kv in sample_pairs:
+        oc = oracle_cache(qo, K[b:b + 1, kv:kv + 1], V[b:b + 1, kv:kv + 1], vb, [N])
+        rows = cache.rows(b, kv)
+        for name, key in (("k_idx", "k_idx"), ("k_signs", "k_signs"), ("k_norms", "k_norms"),
+                          ("v_q", "v_q"), ("v_params", "v_params")):
+            src = oc[key][0, 0]
+            if src.dtype == np.uint16:
+                src = src.view(np.int16)
+            getattr(cache, name)[rows][:N].copy_(torch.from_numpy(np.ascontiguousarray(src)).reshape(
+                getattr(cache, name)[rows][:N].shape))
+        pairs_oc = oc
+        pairs_oc["len"] = np.array([N])
+        heads = list(range(kv * G, (kv + 1) * G))
+        out, _, _ = run_decode(qg, cache, Q, torch.bfloat16, out_dtype)
+        ref, _ = O.decode_attention(qo, pairs_oc, Q[b:b + 1, heads].astype(np.float64),
+                                    head_map=np.zeros(G, dtype=int), value_bits=vb)
+        err = check_attention(out[b, heads], ref[0], out_dtype == torch.bfloat16)
+        print(cfg["name"], b, kv, err)
+    return out
+
+
+def test_decode_full_config_decode_s():
+    """Batch 1, 12/2 GQA, context 32768, 3-bit prod keys, 2-bit values: every head."""
+    _full_decode(2, [(0, 0), (0, 1)], torch.float32)
+
+
+def test_decode_full_config_decode_l():
+    """Batch 8, 28/4 GQA, context 32768 with planted keys; sampled (sequence, KV head)
+    pairs; the planted keys dominate attention for the first head of each group."""
+    out = _full_decode(3, [(0, 0), (7, 3), (3, 1)], torch.bfloat16)
+    assert np.all(np.isfinite(out))
+
+
+def test_decode_stream_steps():
+    """Streaming decode: context 131072, 64/8 GQA, 4-bit prod keys, 4-bit values; each step
+    appends one token per KV head on the GPU, then decodes. Appended rows are checked
+    against the oracle, and the decode after each step against the oracle's cache."""
+    require_cuda()
+    cfg = W.WORKLOADS[5]
+    B, Hq, Hkv, N = 1, cfg["n_q_heads"], cfg["n_kv_heads"], cfg["ctx"]
+    steps = 3
+    K, V, Q, _ = W.decode_inputs(5, B, Hq, Hkv, N, extra_tokens=steps)
+    qo = O.build_quantizer(128, 4, "prod", 0)
+    qg = tq.tq_build_codebook(128, 4, "prod", 0)
+    cap = N + 256
+    cache = tq.KVCache(qg, B, Hkv, cap, value_bits=4, device="cuda:0")
+    tq.tq_append(qg, cache, to_device(K[:, :, :N], torch.bfloat16),
+                 to_device(V[:, :, :N], torch.bfloat16))
+    kv = 5
+    G = Hq // Hkv
+    heads = list(range(kv * G, (kv + 1) * G))
+    oc = oracle_cache(qo, K[:, kv:kv + 1], V[:, kv:kv + 1], 4, [N + steps])
+    rows = cache.rows(0, kv)
+    for name in ("k_idx", "k_signs", "k_norms", "v_q", "v_params"):
+        src = oc[name][0, 0][:N]
+        if src.dtype == np.uint16:
+            src = src.view(np.int16)
+        dst = getattr(cache, name)[rows][:N]
+        dst.copy_(torch.from_numpy(np.ascontiguousarray(src)).reshape(dst.shape))
+    for s in range(steps):
+        tq.tq_append(qg, cache, to_device(K[:, :, N + s:N + s + 1], torch.bfloat16),
+                     to_device(V[:, :, N + s:N + s + 1], torch.bfloat16))
+        r = slice(rows.start + N + s, rows.start + N + s + 1)
+        gp = to_np_planes({"idx": cache.k_idx[r], "signs": cache.k_signs[r], "norms": cache.k_norms[r]})
+        check_key_parity(qo, K[0, kv, N + s:N + s + 1].astype(np.float64), gp)
+        out, _, _ = run_decode(qg, cache, Q, torch.bfloat16, torch.float32)
+        step_oc = dict(oc, len=np.array([N + s + 1]))
+        ref, _ = O.decode_attention(qo, step_oc, Q[:, heads].astype(np.float64),
+                                    head_map=np.zeros(G, dtype=int), value_bits=4)
+        check_attention(out[0, heads], ref[0], False)
