@@ -43,6 +43,10 @@ def parse():
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--no-quantize", action="store_true", help="skip the key-quantize leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", default="all", choices=["all", "decode", "quantize"],
+                    help="run one leg only (small cases for profiling)")
+    ap.add_argument("--quantize-rows", type=int, default=1 << 22, help="rows per layer")
     return ap.parse_args()
 
 
@@ -149,14 +153,18 @@ def sum_over_ranks(x: float, world: int) -> float:
 
 # ------------------------------------------------------------------------------ tq arm
 def run_tq(args):
-    import numpy as np
     import torch
 
     import kv_cache_vector_fwht_b200 as tq
-    import workloads as W
 
     rank, world, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
+    peak, peak_kind = load_peaks()
+    if args.only == "quantize":
+        r = bench_quantize(tq, torch, dev, world, peak, peak_kind, rows=args.quantize_rows)
+        if rank == 0:
+            print(json.dumps({"key_quantize": r}))
+        return
     B, Hq, Hkv, N = CFG["batch"], CFG["n_q_heads"], CFG["n_kv_heads"], CFG["ctx"]
     steps, warm = args.steps, args.warmup
     extra = warm + steps + 8
@@ -218,11 +226,10 @@ def run_tq(args):
     dec_avg_ms = sum(dec_ms) / len(dec_ms)
     mean_len = sum(lens) / len(lens)
     dec_bytes = B * Hkv * mean_len * (KEY_BYTES + VAL_BYTES) + B * Hq * 128 * 2 * 2
-    peak, peak_kind = load_peaks()
     achieved = dec_bytes / (dec_avg_ms / 1e3) / 1e9
 
     # ---- end to end through the public API: host (pinned) inputs in, result out, per step
-    e2e_steps = min(steps, 500)
+    e2e_steps = 0 if args.no_e2e else min(steps, 500)
     kh = Kn[:e2e_steps].cpu().pin_memory()
     vh = Vn[:e2e_steps].cpu().pin_memory()
     qh = Qs[:e2e_steps].cpu().pin_memory()
@@ -244,7 +251,7 @@ def run_tq(args):
         e2e_ms += (time.perf_counter() - t0) * 1e3
     e2e_keys = float(sum(Hq * (N + s + 1) for s in range(e2e_steps)) * B)
     e2e_ms_max = max_over_ranks(e2e_ms, world)
-    e2e_value = sum_over_ranks(e2e_keys, world) / (e2e_ms_max / 1e3)
+    e2e_value = sum_over_ranks(e2e_keys, world) / (e2e_ms_max / 1e3) if e2e_steps else None
 
     result = {
         "metric": "fused-decode keys scored/s (decode-s step: append 1 token per KV head + decode)",
@@ -268,8 +275,9 @@ def run_tq(args):
         "clocks": clk,
         "wall_s_timed_region": t_wall,
     }
-    if not args.no_quantize:
-        result["key_quantize"] = bench_quantize(tq, torch, dev, world, peak, peak_kind)
+    if not args.no_quantize and args.only == "all":
+        result["key_quantize"] = bench_quantize(tq, torch, dev, world, peak, peak_kind,
+                                                rows=args.quantize_rows)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(sample_keys=4096)
     if rank == 0:
@@ -279,11 +287,10 @@ def run_tq(args):
         dist.destroy_process_group()
 
 
-def bench_quantize(tq, torch, dev, world, peak, peak_kind, reps=5):
+def bench_quantize(tq, torch, dev, world, peak, peak_kind, rows=1 << 22, reps=5):
     """Key-quantize throughput: 4 layers x 2^22 bf16 rows (2^24 rows), 3-bit prod, quantizer
     seed = layer, 32 channels at 4x std. Inputs (4 GiB) exceed L2; no flush needed."""
     import workloads as W
-    rows = 1 << 22
     ch = torch.from_numpy(W.outlier_channels(4)).long().to(dev)
     g = torch.Generator(device=dev).manual_seed(4)
     xs, qs, planes = [], [], []
@@ -310,7 +317,8 @@ def bench_quantize(tq, torch, dev, world, peak, peak_kind, reps=5):
     ms = sum(times) / len(times)
     n = 4 * rows
     gbs = n * (256 + KEY_BYTES) / (ms / 1e3) / 1e9
-    return {"rows_per_s": n / (ms / 1e3), "ms_per_2^24_rows": ms, "mode": "prod b=3",
+    return {"rows_per_s": n / (ms / 1e3), "ms_per_pass": ms, "rows_per_pass": n,
+            "mode": "prod b=3",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                          "frac": gbs / peak, "traffic": None,
                          "bytes_per_row": 256 + KEY_BYTES, "kernel": "k_keys_full<prod,3>",
