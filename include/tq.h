@@ -52,7 +52,8 @@ typedef enum {
   TQ_ECAPACITY = -3,     /* cache would overflow: len + n_tokens > capacity */
   TQ_ENOMEM = -4,        /* host or device allocation failed (tq_build_codebook only) */
   TQ_ECUDA = -5,         /* a CUDA runtime call or kernel launch failed */
-  TQ_ETIMEOUT = -6       /* reserved: a bounded device wait gave up */
+  TQ_ETIMEOUT = -6,      /* reserved: a bounded device wait gave up */
+  TQ_ETOOLARGE = -7      /* needs more scratch than tq_decode_attention_noalloc holds */
 } tq_status;
 
 enum { TQ_MODE_MSE = 0, TQ_MODE_PROD = 1, TQ_MODE_GROUPED = 2 };
@@ -189,6 +190,29 @@ tq_status tq_decode_attention(const tq_quantizer* q, const tq_kv_cache* cache,
                               void* out_dev, int out_dtype,
                               float* scores_dev, int64_t scores_ld,
                               void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/* tq_decode_attention without a workspace argument, for callers that cannot allocate
+ * device memory: for example a plain C host with no device allocator of its own, or a
+ * serving loop that must not call cudaMalloc on its hot path (cudaMalloc can synchronize
+ * the device and its latency is unbounded). The paper has no counterpart; this is a
+ * convenience of the library.
+ *
+ * The scratch the decode kernel needs (per-split partial results and split counters)
+ * lives in one file-scope device array of TQ_NOALLOC_SCRATCH_BYTES (16 MiB) that every
+ * GPU loading the library holds until the process exits. Problems whose scratch
+ * (tq_decode_workspace_bytes) exceeds it return TQ_ETOOLARGE and launch nothing.
+ * The first call on a device looks up the array's device address (once per device, with
+ * that device current); make that first call before any stream capture. Each call clears
+ * the split counters it uses (an async memset on `stream`) and allocates nothing. All
+ * calls share the one array: calls whose kernels overlap on the GPU (other streams, other
+ * host threads) race on it and must be serialised by the caller. Arguments and results are
+ * otherwise exactly those of tq_decode_attention. */
+#define TQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+tq_status tq_decode_attention_noalloc(const tq_quantizer* q, const tq_kv_cache* cache,
+                                      const void* q_dev, int q_dtype, int n_q_heads,
+                                      const int32_t* head_map, float sm_scale,
+                                      void* out_dev, int out_dtype,
+                                      float* scores_dev, int64_t scores_ld, void* stream);
 
 const char* tq_status_string(tq_status s);
 int tq_abi_version(void);

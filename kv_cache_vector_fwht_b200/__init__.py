@@ -20,15 +20,17 @@ if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is not built; run `python -m kv_cache_vector_fwht_b200.build`")
 _lib = ctypes.CDLL(LIB_PATH)
 
-TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ECAPACITY, TQ_ENOMEM, TQ_ECUDA, TQ_ETIMEOUT = \
-    0, -1, -2, -3, -4, -5, -6
+TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ECAPACITY, TQ_ENOMEM, TQ_ECUDA, TQ_ETIMEOUT, TQ_ETOOLARGE = \
+    0, -1, -2, -3, -4, -5, -6, -7
+TQ_NOALLOC_SCRATCH_BYTES = 16 << 20
 MODES = {"mse": 0, "prod": 1, "grouped": 2}
 TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 D = 128
 
 EXPORTED = ["tq_build_codebook", "tq_free", "tq_key_layout", "tq_host_tables",
             "tq_quantize_keys", "tq_quantize_values", "tq_append", "tq_decode_workspace_bytes",
-            "tq_decode_attention", "tq_status_string", "tq_abi_version"]
+            "tq_decode_attention", "tq_decode_attention_noalloc", "tq_status_string",
+            "tq_abi_version"]
 
 
 class KeyLayout(ctypes.Structure):
@@ -77,6 +79,10 @@ _lib.tq_decode_attention.argtypes = [c_void_p, POINTER(KVCacheDesc), c_void_p, c
                                      POINTER(c_int32), c_float, c_void_p, c_int, c_void_p,
                                      c_int64, c_void_p, c_size_t, c_void_p]
 _lib.tq_decode_attention.restype = c_int
+_lib.tq_decode_attention_noalloc.argtypes = [c_void_p, POINTER(KVCacheDesc), c_void_p, c_int,
+                                             c_int, POINTER(c_int32), c_float, c_void_p, c_int,
+                                             c_void_p, c_int64, c_void_p]
+_lib.tq_decode_attention_noalloc.restype = c_int
 _lib.tq_status_string.argtypes = [c_int]
 _lib.tq_status_string.restype = ctypes.c_char_p
 _lib.tq_abi_version.argtypes = []
@@ -295,3 +301,19 @@ def tq_decode_attention(q: Quantizer, cache: KVCache, query, out=None, workspace
                                     _dtype_code(out) if out is not None else TQ_F32,
                                     _ptr(scores), sld, _ptr(workspace), wbytes, _stream(stream)),
            "tq_decode_attention")
+
+
+def tq_decode_attention_noalloc(q: Quantizer, cache: KVCache, query, out=None, head_map=None,
+                                sm_scale: float = 0.0, scores=None, stream=None) -> None:
+    """tq_decode_attention without a workspace: for callers that cannot allocate device
+    memory (the library's built-in scratch array is used instead; see tq.h). Raises
+    TQError(TQ_ETOOLARGE) when the problem needs more scratch than the array holds."""
+    assert query.is_contiguous() and query.dim() == 3
+    hq = query.shape[1]
+    hm = (c_int32 * hq)(*[int(v) for v in head_map]) if head_map is not None else None
+    sld = scores.shape[2] if scores is not None else 0
+    _check(_lib.tq_decode_attention_noalloc(q.handle, ctypes.byref(cache.desc), _ptr(query),
+                                            _dtype_code(query), hq, hm, sm_scale, _ptr(out),
+                                            _dtype_code(out) if out is not None else TQ_F32,
+                                            _ptr(scores), sld, _stream(stream)),
+           "tq_decode_attention_noalloc")

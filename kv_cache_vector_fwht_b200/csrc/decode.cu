@@ -22,6 +22,7 @@
 // the last CTA of a (sequence, head group) to finish merges all partials (no spinning).
 #include <cfloat>
 #include <cmath>
+#include <mutex>
 
 #include "tq_device.cuh"
 #include "tq_internal.h"
@@ -607,6 +608,50 @@ tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* c, const void*
     case 3 * 8 + 4: return run_decode<3, 4>(a, grid, st);
     default: return TQ_EUNSUPPORTED;
   }
+}
+
+// ---------------------------------------------------------------------------------------
+// Decode without a caller workspace: the partials and split counters live in this file-scope
+// device array (TQ_NOALLOC_SCRATCH_BYTES, held by every GPU that loads the library until the
+// process exits). Host code cannot use the array's name as a device address; its address
+// is looked up once per device with cudaGetSymbolAddress, with that device current.
+// ---------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[TQ_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+}  // namespace
+
+tq_status launch_decode_noalloc(const tq_quantizer* q, const tq_kv_cache* c, const void* qv,
+                                int q_dtype, int n_q_heads, const int32_t* head_map,
+                                float sm_scale, void* out, int out_dtype, float* scores,
+                                int64_t scores_ld, cudaStream_t st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TQ_ECUDA;
+  void* base = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (g_scratch_addr[dev] == nullptr) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+        return TQ_ECUDA;
+      g_scratch_addr[dev] = p;
+    }
+    base = g_scratch_addr[dev];
+  }
+  const size_t need = decode_workspace_bytes(c->batch, n_q_heads, c->capacity);
+  if (need > TQ_NOALLOC_SCRATCH_BYTES) return TQ_ETOOLARGE;
+  // the split counters must start at zero; earlier calls leave their last contents here
+  const size_t parts = static_cast<size_t>(c->batch) * n_q_heads * max_splits_for(c->capacity) *
+                       kPartStride * sizeof(float);
+  const size_t ctr_off = ((parts + 255) / 256) * 256;
+  const size_t ctr_bytes = static_cast<size_t>(c->batch) * n_q_heads * sizeof(int);
+  if (cudaMemsetAsync(static_cast<unsigned char*>(base) + ctr_off, 0, ctr_bytes, st) != cudaSuccess)
+    return TQ_ECUDA;
+  return launch_decode(q, c, qv, q_dtype, n_q_heads, head_map, sm_scale, out, out_dtype, scores,
+                       scores_ld, base, need, st);
 }
 
 }  // namespace tq

@@ -80,6 +80,7 @@ const char* tq_status_string(tq_status s) {
     case TQ_ENOMEM: return "out of memory";
     case TQ_ECUDA: return "CUDA error";
     case TQ_ETIMEOUT: return "device wait timed out";
+    case TQ_ETOOLARGE: return "problem exceeds the built-in decode scratch";
   }
   return "unknown status";
 }
@@ -238,6 +239,36 @@ tq_status tq_decode_workspace_bytes(const tq_kv_cache* c, int n_q_heads, size_t*
   return TQ_OK;
 }
 
+// Argument checks of the no-workspace decode entry point (the same as tq_decode_attention's
+// checks apart from the workspace).
+static tq_status check_decode_args(const tq_quantizer* q, const tq_kv_cache* c, const void* qv,
+                                   int q_dtype, int n_q_heads, const int32_t* head_map,
+                                   void* out, int out_dtype, float* scores, int64_t scores_ld) {
+  if (!q) return TQ_EINVAL;
+  if (q->mode != TQ_MODE_PROD) return TQ_EUNSUPPORTED;
+  tq_status st = check_cache(q, c);
+  if (st != TQ_OK) return st;
+  if (n_q_heads <= 0 || n_q_heads > 512) return TQ_EINVAL;
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_EUNSUPPORTED;
+  if (!qv || !aligned16(qv)) return TQ_EINVAL;
+  if (head_map) {
+    for (int h = 0; h < n_q_heads; ++h)
+      if (head_map[h] < 0 || head_map[h] >= c->n_kv_heads) return TQ_EINVAL;
+  } else if (n_q_heads % c->n_kv_heads != 0) {
+    return TQ_EINVAL;
+  }
+  if (c->value_bits != 0) {
+    if (!out || !aligned16(out)) return TQ_EINVAL;
+    if (out_dtype != TQ_F32 && out_dtype != TQ_BF16) return TQ_EUNSUPPORTED;
+  } else if (out) {
+    return TQ_EINVAL;
+  }
+  int max_len = 0;
+  for (int b = 0; b < c->batch; ++b) max_len = c->len_host[b] > max_len ? c->len_host[b] : max_len;
+  if (scores && scores_ld < max_len) return TQ_EINVAL;
+  return TQ_OK;
+}
+
 tq_status tq_decode_attention(const tq_quantizer* q, const tq_kv_cache* c, const void* qv,
                               int q_dtype, int n_q_heads, const int32_t* head_map, float sm_scale,
                               void* out, int out_dtype, float* scores, int64_t scores_ld,
@@ -268,6 +299,18 @@ tq_status tq_decode_attention(const tq_quantizer* q, const tq_kv_cache* c, const
   if (workspace_bytes < decode_workspace_bytes(c->batch, n_q_heads, c->capacity)) return TQ_EINVAL;
   return launch_decode(q, c, qv, q_dtype, n_q_heads, head_map, sm_scale, out, out_dtype, scores,
                        scores_ld, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+tq_status tq_decode_attention_noalloc(const tq_quantizer* q, const tq_kv_cache* c,
+                                      const void* qv, int q_dtype, int n_q_heads,
+                                      const int32_t* head_map, float sm_scale, void* out,
+                                      int out_dtype, float* scores, int64_t scores_ld,
+                                      void* stream) {
+  const tq_status st = check_decode_args(q, c, qv, q_dtype, n_q_heads, head_map, out, out_dtype,
+                                         scores, scores_ld);
+  if (st != TQ_OK) return st;
+  return launch_decode_noalloc(q, c, qv, q_dtype, n_q_heads, head_map, sm_scale, out, out_dtype,
+                               scores, scores_ld, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -85,6 +85,11 @@ tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* cache, const v
                         void* out, int out_dtype, float* scores, int64_t scores_ld,
                         void* workspace, size_t workspace_bytes, cudaStream_t st);
 
+tq_status launch_decode_noalloc(const tq_quantizer* q, const tq_kv_cache* cache, const void* qv,
+                                int q_dtype, int n_q_heads, const int32_t* head_map,
+                                float sm_scale, void* out, int out_dtype, float* scores,
+                                int64_t scores_ld, cudaStream_t st);
+
 int sm_count(int device);
 
 }  // namespace tq
