@@ -122,7 +122,10 @@ def _dtype_code(t) -> int:
 def _stream(stream) -> int | None:
     import torch
     if stream is None:
-        return torch.cuda.current_stream().cuda_stream
+        try:   # raw handle of the current stream without building a Stream object
+            return torch._C._cuda_getCurrentRawStream(torch.cuda.current_device())
+        except AttributeError:
+            return torch.cuda.current_stream().cuda_stream
     if isinstance(stream, int):
         return stream
     return stream.cuda_stream

@@ -221,6 +221,11 @@ tq_status tq_append(const tq_quantizer* q, tq_kv_cache* c, const void* k_new, co
   for (int b = 0; b < c->batch; ++b)
     if (static_cast<int64_t>(c->len_host[b]) + n_tokens > c->capacity) return TQ_ECAPACITY;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (append_fused_ok(q, c, n_tokens)) {
+    if ((st = launch_append_fused(q, c, k_new, v_new, dtype, n_tokens, s)) != TQ_OK) return st;
+    for (int b = 0; b < c->batch; ++b) c->len_host[b] += n_tokens;
+    return TQ_OK;
+  }
   const int64_t rows = static_cast<int64_t>(c->batch) * c->n_kv_heads * n_tokens;
   const RowMap map{c->len_dev, c->n_kv_heads, n_tokens, c->capacity};
   if ((st = launch_quantize_keys(q, k_new, dtype, rows, kD, c->keys, map, s)) != TQ_OK) return st;

@@ -72,6 +72,13 @@ tq_status launch_quantize_values(const void* v, int dtype, int64_t n_rows, int64
                                  tq_value_planes out, RowMap map, cudaStream_t st);
 tq_status launch_advance_len(int32_t* len, int batch, int n, cudaStream_t st);
 
+// Fused append of a few tokens (mse / prod keys + values + lengths in one launch).
+constexpr int kMaxAppendBatch = 64;
+constexpr int kMaxAppendRows = 64;
+bool append_fused_ok(const tq_quantizer* q, const tq_kv_cache* c, int n_tokens);
+tq_status launch_append_fused(const tq_quantizer* q, tq_kv_cache* c, const void* k_new,
+                              const void* v_new, int dtype, int n_tokens, cudaStream_t st);
+
 struct DecodePlan {
   int n_groups;          // CTA head groups over all KV heads
   int n_splits;          // context splits per (sequence, head group)

@@ -9,7 +9,9 @@ noise). Where a row took an exempt alternative (a neighbouring code or norm), it
 signs are checked against the oracle's signs for that alternative: the alternative is one
 of the two values the oracle itself accepts, so it is a valid result, not a new input.
 Scores: |ds| <= 1e-3 max(|s_ref|, ||q|| n16 / sqrt(d)). Attention: fp32 output within
-2e-3 max-abs; bf16 output within one bf16 ulp of the oracle's bf16-rounded value.
+2e-3 max-abs; bf16 output within 2e-3 of the oracle's bf16-rounded value, or within one bf16
+ulp of it where that ulp is larger (|out| >= 0.25: a half-ulp of bf16 there already exceeds
+what an fp32 result can be held to).
 """
 from __future__ import annotations
 
@@ -123,7 +125,8 @@ def check_attention(gpu: np.ndarray, ref: np.ndarray, bf16: bool):
         _, e = np.frexp(rb)
         ulp = np.where(rb != 0, np.ldexp(1.0, e - 8), 2.0 ** -133)   # 8 significant bits
         err = np.abs(gpu - rb)
-        assert np.all(err <= ulp), f"bf16 output off by more than 1 ulp: {np.max(err / ulp)}"
+        tol = np.maximum(ulp, 2e-3)
+        assert np.all(err <= tol), f"bf16 output error {np.max(err / tol)} x tolerance"
         return float(np.max(np.abs(gpu - ref)))
     err = float(np.max(np.abs(gpu - ref))) if gpu.size else 0.0
     assert err <= 2e-3, f"attention max-abs error {err}"
