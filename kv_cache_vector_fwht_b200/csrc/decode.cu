@@ -622,45 +622,53 @@ k_decode(const __grid_constant__ DecodeArgs a) {
   __syncthreads();
   if (!sLast) return;
   __threadfence();
-  // every warp folds splits s = warp, warp + 8, ... for all heads against the global maximum
-  // (independent L2 loads, no dependent chain), then warps are summed through shared memory
-  float* sC = reinterpret_cast<float*>(tiles);  // [warp][head][kPartStride]
-  for (int h = 0; h < nh; ++h) {
-    const int hq = a.g_heads[grp][h];
+  // one warp per head, heads in parallel: lanes read the split maxima and sums (lane = split),
+  // then the weighted partial outputs are loaded 16 splits at a time (independent loads)
+  if (warp < nh) {
+    const int h = warp, hq = a.g_heads[grp][h];
     const float* base = a.part + (static_cast<int64_t>(b) * a.n_q_heads + hq) * a.n_splits * kPartStride;
     float mloc = -INFINITY;
     for (int s = lane; s < a.n_splits; s += 32) mloc = fmaxf(mloc, __ldcg(base + s * kPartStride));
     const float M = warp_max(mloc);
-    float Lw = 0.f, O[4] = {0.f, 0.f, 0.f, 0.f};
-    if (M != -INFINITY) {
-#pragma unroll 4
-      for (int s = warp; s < a.n_splits; s += 8) {
-        const float* src = base + s * kPartStride;
-        const float ms = __ldcg(src);
-        const float lsv = __ldcg(src + 1);
-        const float4 ov = __ldcg(reinterpret_cast<const float4*>(src + 4 + 4 * lane));
-        const float f = ms == -INFINITY ? 0.f : exp2f(ms - M);
-        Lw = fmaf(f, lsv, Lw);
-        O[0] = fmaf(f, ov.x, O[0]);
-        O[1] = fmaf(f, ov.y, O[1]);
-        O[2] = fmaf(f, ov.z, O[2]);
-        O[3] = fmaf(f, ov.w, O[3]);
-      }
-    }
-    float* dst = sC + (warp * kMaxHeads + h) * kPartStride;
-    if (lane == 0) dst[1] = Lw;
-    *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = make_float4(O[0], O[1], O[2], O[3]);
-  }
-  __syncthreads();
-  if (warp < nh) {
-    const int h = warp, hq = a.g_heads[grp][h];
     float Lsum = 0.f, O[4] = {0.f, 0.f, 0.f, 0.f};
+    if (M != -INFINITY) {
+      for (int s0 = 0; s0 < a.n_splits; s0 += 32) {
+        const int s = s0 + lane;
+        float f = 0.f;
+        if (s < a.n_splits) {
+          const float ms = __ldcg(base + s * kPartStride);
+          const float lsv = __ldcg(base + s * kPartStride + 1);
+          if (ms != -INFINITY) {
+            f = exp2f(ms - M);
+            Lsum = fmaf(f, lsv, Lsum);
+          }
+        }
+        const int cnt = min(32, a.n_splits - s0);
+        const float* blk = base + s0 * kPartStride + 4 + 4 * lane;
+        int j = 0;
+        for (; j + 16 <= cnt; j += 16) {
+          float4 ov[16];
 #pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      const float* src = sC + (w * kMaxHeads + h) * kPartStride;
-      Lsum += src[1];
-      const float4 ov = *reinterpret_cast<const float4*>(src + 4 + 4 * lane);
-      O[0] += ov.x; O[1] += ov.y; O[2] += ov.z; O[3] += ov.w;
+          for (int u = 0; u < 16; ++u) ov[u] = __ldcg(reinterpret_cast<const float4*>(blk + (j + u) * kPartStride));
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const float fj = __shfl_sync(kFull, f, j + u);
+            O[0] = fmaf(fj, ov[u].x, O[0]);
+            O[1] = fmaf(fj, ov[u].y, O[1]);
+            O[2] = fmaf(fj, ov[u].z, O[2]);
+            O[3] = fmaf(fj, ov[u].w, O[3]);
+          }
+        }
+        for (; j < cnt; ++j) {
+          const float fj = __shfl_sync(kFull, f, j);
+          const float4 ov = __ldcg(reinterpret_cast<const float4*>(blk + j * kPartStride));
+          O[0] = fmaf(fj, ov.x, O[0]);
+          O[1] = fmaf(fj, ov.y, O[1]);
+          O[2] = fmaf(fj, ov.z, O[2]);
+          O[3] = fmaf(fj, ov.w, O[3]);
+        }
+      }
+      Lsum = warp_sum(Lsum);
     }
     const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
     const int64_t orow = (static_cast<int64_t>(b) * a.n_q_heads + hq) * kD + 4 * lane;
@@ -766,11 +774,11 @@ tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* c, const void*
   for (int b = 0; b < c->batch; ++b) max_len = c->len_host[b] > max_len ? c->len_host[b] : max_len;
   if (max_len == 0 && out == nullptr) return TQ_OK;
 
-  // split count: minimise waves x (tokens per split + per-CTA set-up); the 1- and 2-bit MSE
-  // kernels fit two CTAs per SM, the 3-bit one a single CTA
+  // split count: minimise (CTAs per SM) x (tokens per split + per-CTA set-up) + the final
+  // combine; CTAs sharing an SM share its issue slots, so they count as serial work
   int dev = 0;
   cudaGetDevice(&dev);
-  const int sms = sm_count(dev) * (q->bits - 1 == 3 ? 1 : 2);
+  const int sms = sm_count(dev);
   const int pairs = c->batch * n_groups;
   const int cap_splits = max_splits_for(c->capacity);
   int best = 1;
@@ -781,7 +789,7 @@ tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* c, const void*
     const int used = (max_len + tps - 1) / tps;
     if (used != s) continue;
     const double waves = std::ceil(static_cast<double>(pairs) * s / sms);
-    const double cost = waves * (tps + 256.0);
+    const double cost = waves * (tps + 256.0) + (s > 1 ? 4.0 * s : 0.0);
     if (cost < best_cost - 1e-9) { best_cost = cost; best = s; }
   }
   a.n_splits = best;
