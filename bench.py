@@ -314,6 +314,7 @@ def bench_quantize(tq, torch, dev, world, peak, peak_kind, rows=1 << 22, reps=5)
         e1.record(st)
         e1.synchronize()
         times.append(e0.elapsed_time(e1))
+    tq.tq_sync_status()
     ms = sum(times) / len(times)
     n = 4 * rows
     gbs = n * (256 + KEY_BYTES) / (ms / 1e3) / 1e9
@@ -321,7 +322,7 @@ def bench_quantize(tq, torch, dev, world, peak, peak_kind, rows=1 << 22, reps=5)
             "mode": "prod b=3",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                          "frac": gbs / peak, "traffic": None,
-                         "bytes_per_row": 256 + KEY_BYTES, "kernel": "k_keys_full<prod,3>",
+                         "bytes_per_row": 256 + KEY_BYTES, "kernel": "k_keys_prod_tc<2>",
                          "peak_kind": f"{peak_kind} (hbm_gbs, burst)"}}
 
 

@@ -52,7 +52,7 @@ typedef enum {
   TQ_ECAPACITY = -3,     /* cache would overflow: len + n_tokens > capacity */
   TQ_ENOMEM = -4,        /* host or device allocation failed (tq_build_codebook only) */
   TQ_ECUDA = -5,         /* a CUDA runtime call or kernel launch failed */
-  TQ_ETIMEOUT = -6,      /* reserved: a bounded device wait gave up */
+  TQ_ETIMEOUT = -6,      /* a bounded device wait gave up (tq_sync_status) */
   TQ_ETOOLARGE = -7      /* needs more scratch than tq_decode_attention_noalloc holds */
 } tq_status;
 
@@ -213,6 +213,14 @@ tq_status tq_decode_attention_noalloc(const tq_quantizer* q, const tq_kv_cache* 
                                       const int32_t* head_map, float sm_scale,
                                       void* out_dev, int out_dtype,
                                       float* scores_dev, int64_t scores_ld, void* stream);
+
+/* Wait for `stream` (cudaStream_t as void*, NULL = legacy default stream) and report whether
+ * any library kernel since the previous call gave up one of its bounded device waits (an
+ * mbarrier wait on a bulk copy or a tensor-core product, limit 2 s): TQ_ETIMEOUT if so (the
+ * flag is then cleared, and the outputs of that kernel are incomplete), TQ_ECUDA if the
+ * stream reports a CUDA error, else TQ_OK. The flag is per process and device, shared by
+ * all streams. */
+tq_status tq_sync_status(void* stream);
 
 const char* tq_status_string(tq_status s);
 int tq_abi_version(void);

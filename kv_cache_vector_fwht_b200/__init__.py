@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libtq.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is not built; run `python -m kv_cache_vector_fwht_b200.build`")
+    raise ImportError(f"{LIB_PATH} is not built; run `python kv_cache_vector_fwht_b200/build.py`")
 _lib = ctypes.CDLL(LIB_PATH)
 
 TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ECAPACITY, TQ_ENOMEM, TQ_ECUDA, TQ_ETIMEOUT, TQ_ETOOLARGE = \
@@ -29,8 +29,8 @@ D = 128
 
 EXPORTED = ["tq_build_codebook", "tq_free", "tq_key_layout", "tq_host_tables",
             "tq_quantize_keys", "tq_quantize_values", "tq_append", "tq_decode_workspace_bytes",
-            "tq_decode_attention", "tq_decode_attention_noalloc", "tq_status_string",
-            "tq_abi_version"]
+            "tq_decode_attention", "tq_decode_attention_noalloc", "tq_sync_status",
+            "tq_status_string", "tq_abi_version"]
 
 
 class KeyLayout(ctypes.Structure):
@@ -87,6 +87,8 @@ _lib.tq_status_string.argtypes = [c_int]
 _lib.tq_status_string.restype = ctypes.c_char_p
 _lib.tq_abi_version.argtypes = []
 _lib.tq_abi_version.restype = c_int
+_lib.tq_sync_status.argtypes = [c_void_p]
+_lib.tq_sync_status.restype = c_int
 
 
 class TQError(RuntimeError):
@@ -106,6 +108,12 @@ def tq_status_string(status: int) -> str:
 
 def tq_abi_version() -> int:
     return _lib.tq_abi_version()
+
+
+def tq_sync_status(stream=None) -> None:
+    """Wait for `stream` and raise TQError(TQ_ETIMEOUT) if a library kernel gave up a bounded
+    device wait since the previous call (TQ_ECUDA on a CUDA error)."""
+    _check(_lib.tq_sync_status(_stream(stream)), "tq_sync_status")
 
 
 def _dtype_code(t) -> int:

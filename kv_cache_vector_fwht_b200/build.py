@@ -1,4 +1,4 @@
-"""Build libtq.so in-tree for sm_100a with nvcc (python -m kv_cache_vector_fwht_b200.build).
+"""Build libtq.so in-tree for sm_100a with nvcc (python kv_cache_vector_fwht_b200/build.py).
 
 Objects go to _build/ at the repository root; the shared library lands next to this file so
 that it travels with the source tree. Rebuilds only sources newer than their objects.
@@ -17,7 +17,7 @@ OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libtq.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
-SOURCES = ["tq_api.cu", "quantize.cu", "decode.cu", "append.cu", "tq_host.cpp"]
+SOURCES = ["tq_api.cu", "quantize.cu", "keys_tc.cu", "decode.cu", "append.cu", "tq_host.cpp"]
 HEADERS = ["tq_internal.h", "tq_device.cuh", os.path.join("..", "..", "include", "tq.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O3",

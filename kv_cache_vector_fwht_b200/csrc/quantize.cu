@@ -420,6 +420,7 @@ tq_status dispatch_keys(int mode, int bits, const KeyArgs& a, cudaStream_t st) {
 tq_status launch_quantize_keys(const tq_quantizer* q, const void* x, int dtype, int64_t n_rows,
                                int64_t ld, tq_key_planes out, RowMap map, cudaStream_t st) {
   if (n_rows == 0) return TQ_OK;
+  if (keys_tc_ok(q, dtype)) return launch_keys_tc(q, x, n_rows, ld, out, map, st);
   KeyArgs a{x, n_rows, ld, q->dev, out.idx, out.signs, out.norms, map};
   return dtype == TQ_F32 ? dispatch_keys<true>(q->mode, q->bits, a, st)
                          : dispatch_keys<false>(q->mode, q->bits, a, st);

@@ -71,6 +71,10 @@ extern "C" {
 
 int tq_abi_version(void) { return TQ_ABI_VERSION; }
 
+tq_status tq_sync_status(void* stream) {
+  return take_device_error(static_cast<cudaStream_t>(stream));
+}
+
 const char* tq_status_string(tq_status s) {
   switch (s) {
     case TQ_OK: return "ok";

@@ -71,6 +71,12 @@ tq_status launch_quantize_keys(const tq_quantizer* q, const void* x, int dtype, 
 tq_status launch_quantize_values(const void* v, int dtype, int64_t n_rows, int64_t ld, int bits,
                                  tq_value_planes out, RowMap map, cudaStream_t st);
 tq_status launch_advance_len(int32_t* len, int batch, int n, cudaStream_t st);
+// prod-mode bf16 keys with the QJL projection on tcgen05 tensor cores
+bool keys_tc_ok(const tq_quantizer* q, int dtype);
+tq_status launch_keys_tc(const tq_quantizer* q, const void* x, int64_t n_rows, int64_t ld,
+                         tq_key_planes out, RowMap map, cudaStream_t st);
+// Synchronise `st`; TQ_ETIMEOUT (and clear the flag) if a kernel gave up a bounded wait.
+tq_status take_device_error(cudaStream_t st);
 
 // Fused append of a few tokens (mse / prod keys + values + lengths in one launch).
 constexpr int kMaxAppendBatch = 64;
