@@ -1,6 +1,5 @@
 // prod-mode key quantization of bf16 rows with the QJL projection on the 5th-generation
-// tensor cores (sm_100a: tcgen05.mma, operands and accumulator in tensor memory / shared
-// memory).
+// tensor cores (sm_100a: TMA, tcgen05.mma, tensor memory).
 //
 // What is computed (tqlite README: rotation.py, codebook.py, prod.py; Implementing TurboQuant
 // (part 5), algorithm overview; TurboQuant bit-packing article sections 2-4), per row x:
@@ -9,18 +8,30 @@
 //   QJL bits [(S_rot rho)_j >= 0] (= [(S r)_j >= 0] with S = S_rot Pi).
 //
 // Work split. A CTA of four warps owns a tile of 128 rows: thread i owns row i of the tile,
-// which is also lane i of the tensor-memory accumulator. Rows arrive in shared memory by
-// bulk copies (double-buffered, one tile ahead); the norm, the rotation (seven butterfly
-// stages in registers), the codebook decisions and the residual run on the CUDA cores. The
-// residual, scaled by a power of two and split into fp16 hi + lo halves, is written to tensor
-// memory as the A operand (128 x 256, K = hi then lo); S_rot, fp16-exact, sits in shared
-// memory as the B operand. Sixteen m128 n128 k16 MMAs accumulate D = [hi | lo] [S | S]^T in
-// fp32 (hi and lo products are exact in fp32, so D carries the fp32 accuracy of S_rot rho).
-// The sign bits of D are taken while the next tile is rotated.
+// which is also lane i of its tensor-memory (TMEM) region. Per tile:
+//   1. TMA brings the 128 x 256 B tile into shared memory (two 64-column boxes, 128-byte
+//      swizzle, double-buffered one tile ahead).
+//   2. Each thread reads its row, applies the rotation signs, takes the norm and runs all
+//      seven butterfly stages of the Hadamard transform in registers.
+//   3. It takes the sign bits of the previous tile's QJL product from the accumulator
+//      columns, then parks its transformed row in those same columns.
+//   4. A rolled loop over column groups reloads the row from TMEM, makes the codebook
+//      decisions, packs the indices and writes the residual -- scaled by a power of two and
+//      split into fp16 hi + lo halves -- into TMEM as the MMA's A operand (128 x 256, K = hi
+//      then lo).
+//   5. When all 128 threads have arrived on an mbarrier, one thread issues sixteen m128 n128
+//      k16 tcgen05.mma with S_rot (fp16-exact, shared memory, B operand) and commits them to
+//      a second mbarrier: D = [hi | lo] [S | S]^T in fp32. The products of fp16 values are
+//      exact in fp32, so D carries the fp32 accuracy of S_rot rho.
+// No CTA-wide barrier sits inside the tile loop; every wait is an mbarrier wait bounded in
+// time, after which the kernel records an error (tq_sync_status) and skips further work.
 //
-// Registers hold the row as 64 fp32 pairs (y_p, y_{p + 64}); the K order of both operands is
-// permuted to match (k' = 2p holds element p, k' = 2p + 1 element p + 64), which leaves the
-// product unchanged.
+// Registers hold the row as 64 fp32 pairs (y_p, y_{p + 64}); the K order of both MMA
+// operands is permuted to match (k' = 2p holds element p, k' = 2p + 1 element p + 64), which
+// leaves the product unchanged.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "tq_device.cuh"
 #include "tq_internal.h"
 
@@ -28,17 +39,18 @@ namespace tq {
 namespace {
 
 constexpr int kTile = 128;             // rows per tile = MMA M = TMEM lanes
-constexpr int kXStride = 272;          // bytes per staged row (256 + 16: conflict-free reads)
-constexpr int kXBuf = kTile * kXStride;
+constexpr int kXBuf = kTile * 256;     // one staged tile (two 16 KB swizzled boxes)
 constexpr int kBBytes = kD * kD * 2;   // S_rot operand
-constexpr int kSmemBytes = kBBytes + 2 * kXBuf + 256;
+constexpr int kMaskOff = kBBytes + 2 * kXBuf;
+constexpr int kCodeOff = kMaskOff + 256;
+constexpr int kSmemBytes = kCodeOff + 16 * kTile * 4;
 constexpr uint32_t kTmemCols = 256;    // D: columns [0, 128); A: hi [128, 192), lo [192, 256)
 constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr int64_t kChunkRows = int64_t(1) << 30;  // rows per launch (TMA row coordinate is int32)
 
 struct TcKeyArgs {
-  const uint16_t* x;
-  int64_t n_rows;
-  int64_t ld;
+  int64_t n_rows;    // rows of this launch
+  int64_t row_base;  // global index of its first row
   int64_t n_tiles;
   const DevTables* tab;
   uint8_t* idx;
@@ -61,54 +73,71 @@ __device__ __forceinline__ uint32_t h2_bits(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Issue the bulk copies of local tile k into buffer k & 1 (called by warp 0).
-__device__ __forceinline__ void issue_tile(const TcKeyArgs& a, uint8_t* sX, uint64_t* bar,
-                                           int64_t tile, int lane) {
-  const int64_t r0 = tile * kTile;
-  const int nv = static_cast<int>(a.n_rows - r0 < kTile ? a.n_rows - r0 : kTile);
-  if (lane == 0) mbar_expect_tx(bar, static_cast<uint32_t>(nv) * 256u);
-  __syncwarp();
-  for (int r = lane; r < nv; r += 32)
-    bulk_g2s(sX + r * kXStride, a.x + (r0 + r) * a.ld, 256u, bar);
+// 1.0f if a > b else 0.0f (an exact compare)
+__device__ __forceinline__ float gt_one(float a, float b) {
+  float d;
+  asm("set.gt.f32.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
 }
 
-// Sign bits [D_j >= 0] of this thread's accumulator row, stored as the row's 16-byte plane.
-__device__ __forceinline__ void store_signs(const TcKeyArgs& a, uint32_t tlane, bool valid,
-                                            int64_t row) {
-  uint32_t sg[4] = {0u, 0u, 0u, 0u};
+// Bits [d_i >= 0] of 32 fp32 values taken from their sign bits (a -0 result cannot occur for
+// a nonzero residual; all-zero residual rows are handled by the caller). Byte permutes gather
+// the top bytes of d[m], d[m+8], d[m+16], d[m+24] into one word whose sign bits are then
+// shifted into bit positions m, m + 8, m + 16, m + 24.
+__device__ __forceinline__ uint32_t sign_word(const uint32_t (&d)[32]) {
+  uint32_t acc = 0;
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    uint32_t d[16];
-    tmem_ld16(tlane + 16 * q, d);
-    tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-      sg[q >> 1] |= (__uint_as_float(d[i]) >= 0.f ? 1u : 0u) << (16 * (q & 1) + i);
+  for (int m = 0; m < 8; ++m) {
+    const uint32_t t1 = __byte_perm(d[m], d[m + 8], 0x0073);
+    const uint32_t t2 = __byte_perm(d[m + 16], d[m + 24], 0x0073);
+    const uint32_t g = __byte_perm(t1, t2, 0x5410);
+    const uint32_t sh = m < 7 ? __umulhi(g, 1u << (25 + m)) : g;  // g >> (7 - m)
+    acc |= sh & (0x01010101u << m);
   }
+  return ~acc;
+}
+
+// Sign bits of this thread's accumulator row (its TMEM lane), stored as the row's 16-byte
+// sign plane.
+__device__ __forceinline__ void store_signs(const TcKeyArgs& a, uint32_t tlane, bool valid,
+                                            bool zero_res, int64_t grow) {
+  uint32_t sg[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t d[32];
+    tmem_ld32_sync(tlane + 32 * q, d);
+    sg[q] = sign_word(d);
+  }
+  if (zero_res) sg[0] = sg[1] = sg[2] = sg[3] = 0xffffffffu;  // S_rot 0 = 0 >= 0
   if (valid)
-    *reinterpret_cast<uint4*>(a.sgn + out_row_tc(a.map, row) * 16) =
+    *reinterpret_cast<uint4*>(a.sgn + out_row_tc(a.map, grow) * 16) =
         make_uint4(sg[0], sg[1], sg[2], sg[3]);
 }
 
 template <int MB>
-__global__ void __launch_bounds__(128, 2) k_keys_prod_tc(const __grid_constant__ TcKeyArgs a) {
+__global__ void __launch_bounds__(128, 2)
+    k_keys_prod_tc(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ TcKeyArgs a) {
   constexpr int NL = 1 << MB;
   constexpr int W = storage_width_c(MB);
-  constexpr int IB = kD * W / 8;  // index bytes per row
-  constexpr int NW = IB / 4;      // index words per row
+  constexpr int NW = 4 * W;       // index words per row
+  constexpr int GP = 32 / W;      // pairs per decision group: one index word per half
+  constexpr int NG = 64 / GP;     // decision groups
 
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sB = smem;
   uint8_t* sX = smem + kBBytes;
-  uint32_t* sMask = reinterpret_cast<uint32_t*>(smem + kBBytes + 2 * kXBuf);
+  const uint32_t* sMask = reinterpret_cast<const uint32_t*>(smem + kMaskOff);
+  uint32_t* sCode = reinterpret_cast<uint32_t*>(smem + kCodeOff);
   __shared__ __align__(8) uint64_t bar_x[2];
+  __shared__ __align__(8) uint64_t bar_b;
   __shared__ __align__(8) uint64_t bar_mma;
+  __shared__ __align__(8) uint64_t bar_a;
   __shared__ uint32_t tslot;
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const DevTables* __restrict__ tab = a.tab;
   const int64_t grid = gridDim.x;
-  const int64_t n_local = a.n_tiles > blockIdx.x ? (a.n_tiles - blockIdx.x + grid - 1) / grid : 0;
+  const int64_t n_local = (a.n_tiles - blockIdx.x + grid - 1) / grid;  // grid <= n_tiles
 
   if (warp == 0) {
     tmem_alloc(&tslot, kTmemCols);
@@ -117,37 +146,28 @@ __global__ void __launch_bounds__(128, 2) k_keys_prod_tc(const __grid_constant__
   if (tid == 0) {
     mbar_init(&bar_x[0], 1);
     mbar_init(&bar_x[1], 1);
+    mbar_init(&bar_b, 1);
     mbar_init(&bar_mma, 1);
+    mbar_init(&bar_a, kTile);
     fence_mbar_init();
   }
-  // B operand: S_rot with the permuted K order, canonical K-major no-swizzle layout
-  // (8-row x 16-byte core matrices; K-adjacent core matrices 128 B apart, 8-row groups 2 KB).
-  for (int c = tid; c < kD * 16; c += blockDim.x) {
-    const int j = c >> 4, kc = c & 15;
-    const __half* srow = tab->s_rot + j * kD;
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int p = 4 * kc + i;
-      w[i] = static_cast<uint32_t>(__half_as_ushort(srow[p])) |
-             (static_cast<uint32_t>(__half_as_ushort(srow[p + 64])) << 16);
-    }
-    *reinterpret_cast<uint4*>(sB + (j >> 3) * 2048 + kc * 128 + (j & 7) * 16) =
-        make_uint4(w[0], w[1], w[2], w[3]);
-  }
-  // sign masks for bf16 pairs: word q flips elements 2q (bit 15) and 2q + 1 (bit 31)
-  if (tid < 64) {
-    const int j = 2 * tid;
-    const uint32_t b0 = (tab->sign_bits[j >> 5] >> (j & 31)) & 1u;
-    const uint32_t b1 = (tab->sign_bits[(j + 1) >> 5] >> ((j + 1) & 31)) & 1u;
-    sMask[tid] = (b0 << 15) | (b1 << 31);
-  }
-  fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = tslot;
   const uint32_t tlane = tbase + (static_cast<uint32_t>(warp * 32) << 16);
+
+  if (tid == 0) {
+    mbar_expect_tx(&bar_b, kBBytes + 256);
+    bulk_g2s(sB, tab->s_umma, kBBytes, &bar_b);
+    bulk_g2s(smem + kMaskOff, tab->pair_mask, 256, &bar_b);
+    for (int k = 0; k < 2 && k < n_local; ++k) {
+      const int row0 = static_cast<int>((blockIdx.x + k * grid) * kTile);
+      mbar_expect_tx(&bar_x[k], kXBuf);
+      tma_load_2d(sX + k * kXBuf, &tmap, 0, row0, &bar_x[k]);
+      tma_load_2d(sX + k * kXBuf + kXBuf / 2, &tmap, 64, row0, &bar_x[k]);
+    }
+  }
 
   float thr[NL - 1], cen[NL];
 #pragma unroll
@@ -155,61 +175,49 @@ __global__ void __launch_bounds__(128, 2) k_keys_prod_tc(const __grid_constant__
 #pragma unroll
   for (int k = 0; k < NL; ++k) cen[k] = tab->cent[0][k];
 
-  if (warp == 0) {
-    if (n_local > 0) issue_tile(a, sX, &bar_x[0], blockIdx.x, lane);
-    if (n_local > 1) issue_tile(a, sX + kXBuf, &bar_x[1], blockIdx.x + grid, lane);
-  }
-
   constexpr uint32_t idesc = umma_idesc_f16(kTile, kD);
-  bool failed = false;
-  int64_t prev_row = -1;  // global row of this thread in the previous tile (-1: none)
-  bool prev_valid = false;
+  bool ok = mbar_wait_ns(&bar_b, 0, kWaitNs);
+  int64_t prev_row = 0;
+  bool prev_valid = false, prev_zero = false;
+  const uint32_t sw = static_cast<uint32_t>(tid & 7);  // 128-byte swizzle phase of this row
 
   for (int64_t k = 0; k < n_local; ++k) {
     const int b = static_cast<int>(k & 1);
-    const uint32_t ph = static_cast<uint32_t>((k >> 1) & 1);
     const int64_t tile = blockIdx.x + k * grid;
-    if (!__syncthreads_and(mbar_wait_ns(&bar_x[b], ph, kWaitNs))) {
-      failed = true;
-      break;
-    }
     const int64_t row = tile * kTile + tid;
     const bool valid = row < a.n_rows;
+    if (ok) ok = mbar_wait_ns(&bar_x[b], static_cast<uint32_t>((k >> 1) & 1), kWaitNs);
 
-    // ---- load the row, flip signs, norm; pairs P[p] = (x_p, x_{p+64})
+    // ---- row from shared memory: signs, first butterfly stage, norm.
+    // P[p] = (x_p + x_{p+64}, x_p - x_{p+64}) after the distance-64 stage.
     uint64_t P[64];
-    float ss;
+    uint64_t nacc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) nacc[i] = pk2(0.f, 0.f);
     {
-      const uint8_t* xr = sX + b * kXBuf + tid * kXStride;
-      uint32_t wl[32], wh[32];  // bf16 pairs of elements [0, 64) and [64, 128)
+      const uint8_t* x0 = sX + b * kXBuf + tid * 128;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const uint4 u0 = *reinterpret_cast<const uint4*>(xr + 16 * c);
-        const uint4 u1 = *reinterpret_cast<const uint4*>(xr + 128 + 16 * c);
+        const uint32_t off = (static_cast<uint32_t>(c) ^ sw) << 4;
+        const uint4 u0 = *reinterpret_cast<const uint4*>(x0 + off);
+        const uint4 u1 = *reinterpret_cast<const uint4*>(x0 + kXBuf / 2 + off);
         const uint4 m0 = *reinterpret_cast<const uint4*>(sMask + 4 * c);
         const uint4 m1 = *reinterpret_cast<const uint4*>(sMask + 32 + 4 * c);
-        wl[4 * c + 0] = u0.x ^ m0.x; wl[4 * c + 1] = u0.y ^ m0.y;
-        wl[4 * c + 2] = u0.z ^ m0.z; wl[4 * c + 3] = u0.w ^ m0.w;
-        wh[4 * c + 0] = u1.x ^ m1.x; wh[4 * c + 1] = u1.y ^ m1.y;
-        wh[4 * c + 2] = u1.z ^ m1.z; wh[4 * c + 3] = u1.w ^ m1.w;
-      }
-      uint64_t acc = pk2(0.f, 0.f);
+        const uint32_t wl[4] = {u0.x ^ m0.x, u0.y ^ m0.y, u0.z ^ m0.z, u0.w ^ m0.w};
+        const uint32_t wh[4] = {u1.x ^ m1.x, u1.y ^ m1.y, u1.z ^ m1.z, u1.w ^ m1.w};
 #pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        // elements 2q, 2q + 1 and 64 + 2q, 64 + 2q + 1
-        const float a0 = __uint_as_float(wl[q] << 16), a1 = __uint_as_float(wl[q] & 0xffff0000u);
-        const float b0 = __uint_as_float(wh[q] << 16), b1 = __uint_as_float(wh[q] & 0xffff0000u);
-        const uint64_t e0 = pk2(a0, b0), e1 = pk2(a1, b1);
-        acc = fma2(e0, e0, acc);
-        acc = fma2(e1, e1, acc);
-        // first butterfly stage (distance 64): (x_p + x_{p+64}, x_p - x_{p+64})
-        P[2 * q] = pk2(a0 + b0, a0 - b0);
-        P[2 * q + 1] = pk2(a1 + b1, a1 - b1);
+        for (int i = 0; i < 4; ++i) {
+          const float a0 = __uint_as_float(wl[i] * 65536u), a1 = __uint_as_float(wl[i] & 0xffff0000u);
+          const float b0 = __uint_as_float(wh[i] * 65536u), b1 = __uint_as_float(wh[i] & 0xffff0000u);
+          const int p = 8 * c + 2 * i;
+          P[p] = pk2(a0 + b0, a0 - b0);
+          P[p + 1] = pk2(a1 + b1, a1 - b1);
+          nacc[(2 * i) & 7] = fma2(P[p], P[p], nacc[(2 * i) & 7]);
+          nacc[(2 * i + 1) & 7] = fma2(P[p + 1], P[p + 1], nacc[(2 * i + 1) & 7]);
+        }
       }
-      const float2 s2 = up2(acc);
-      ss = s2.x + s2.y;
     }
-    // ---- remaining butterfly stages on pair indices (distances 1 .. 32)
+    // ---- butterfly stages of distance 1 .. 32 on pair indices
 #pragma unroll
     for (int h = 1; h < 64; h <<= 1) {
 #pragma unroll
@@ -221,112 +229,170 @@ __global__ void __launch_bounds__(128, 2) k_keys_prod_tc(const __grid_constant__
         }
       }
     }
-    const float n = sqrtf(ss);
+    // (a + b)^2 + (a - b)^2 = 2 (a^2 + b^2)
+#pragma unroll
+    for (int i = 1; i < 8; i <<= 1)
+#pragma unroll
+      for (int j = 0; j < 8; j += 2 * i) nacc[j] = add2(nacc[j], nacc[j + i]);
+    const float2 n2 = up2(nacc[0]);
+    const float n = sqrtf((n2.x + n2.y) * 0.5f);
     const __half n16 = __float2half_rn(n);
     const float n16f = __half2float(n16);
 
-    // ---- previous tile: wait for its MMA, take the sign bits of D
+    // ---- previous tile: sign bits of its QJL product
     if (k > 0) {
-      if (!__syncthreads_and(mbar_wait_ns(&bar_mma, static_cast<uint32_t>((k - 1) & 1), kWaitNs))) {
-        failed = true;
-        break;
-      }
+      if (ok) ok = mbar_wait_ns(&bar_mma, static_cast<uint32_t>((k - 1) & 1), kWaitNs);
       tc_fence_after();
-      store_signs(a, tlane, prev_valid, prev_row);
+      store_signs(a, tlane, prev_valid, prev_zero, a.row_base + prev_row);
     }
 
-    // ---- decisions, packed indices, residual, fp16 hi/lo halves into tensor memory
+    // ---- park the transformed row in the accumulator columns (pair p -> columns 2p, 2p + 1)
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      uint32_t r[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float2 v = up2(P[8 * q + i]);
+        r[2 * i] = __float_as_uint(v.x);
+        r[2 * i + 1] = __float_as_uint(v.y);
+      }
+      tmem_st16(tlane + 16 * q, r);
+    }
+    tmem_st_wait();
+
+    // ---- per-row decision tables. Power-of-two scale scl keeps |rho| scl below 2^15
+    // (|rho_j| <= (sqrt(d) + 2.2) n); ncs[k] = -scl RN(n16 C_k), so rho scl = fma(y, scl, ncs).
     float T[NL - 1];
 #pragma unroll
     for (int t = 0; t < NL - 1; ++t) T[t] = n > 0.f ? thr[t] * n : thr[t];
-    // power-of-two scale keeping |rho| * scl below 2^15 (|rho_j| <= (sqrt(d) + 2.2) n)
     const uint32_t ex = (__float_as_uint(n) >> 23) & 0xffu;
     const float scl = __uint_as_float((ex >= 10u ? 264u - ex : 254u) << 23);
+    // The centroid term of code c is ncs[0] + sum_{t < c} dcs[t]: a multiply-add per exact
+    // 0/1 compare (its rounding moves rho by about an ulp, far inside the parity margins).
+    float ncs[NL];
+#pragma unroll
+    for (int t = 0; t < NL; ++t) ncs[t] = -(n16f * cen[t]) * scl;
+    uint64_t dcs2[NL - 1], T2[NL - 1];
+#pragma unroll
+    for (int t = 0; t < NL - 1; ++t) {
+      dcs2[t] = pk2(ncs[t + 1] - ncs[t], ncs[t + 1] - ncs[t]);
+      T2[t] = pk2(T[t], T[t]);
+    }
+    const uint64_t ncs02 = pk2(ncs[0], ncs[0]);
     const uint64_t scl2 = pk2(scl, scl);
-    const uint64_t mn2 = pk2(-n16f, -n16f);
-    uint32_t pk[NW];
+    const uint64_t kSplit2 = pk2(8192.f, 8192.f);  // c = 8192 r + r
+
+    uint64_t racc[4];
 #pragma unroll
-    for (int w = 0; w < NW; ++w) pk[w] = 0u;
-    uint64_t racc = pk2(0.f, 0.f);
+    for (int i = 0; i < 4; ++i) racc[i] = pk2(0.f, 0.f);
+#pragma unroll 1
+    for (int g = 0; g < NG; ++g) {
+      // index words of elements [GP g, GP g + GP) (.x) and +64 (.y), accumulated in fp32 as
+      // exact integers: codes of pairs [0, GP/2) in wa, [GP/2, GP) in wb (each < 2^16)
+      uint64_t wa = pk2(0.f, 0.f), wb = pk2(0.f, 0.f);
+      uint32_t hw[GP], lw[GP];
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      uint32_t hw[8], lw[8];
+      for (int q = 0; q < GP / 8; ++q) {
+        uint32_t yv[16];
+        tmem_ld16_sync(tlane + 2 * GP * g + 16 * q, yv);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int p = 8 * g + i;
-        const float2 y = up2(P[p]);
-        float c2[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float yv = e ? y.y : y.x;
-          const int j = p + 64 * e;
-          uint32_t id = 0;
-          float c = cen[0];
+        for (int i = 0; i < 8; ++i) {
+          const int pi = 8 * q + i;  // pair index within the group
+          // index = number of thresholds below y: each exact 0/1 compare adds 2^(W slot) to
+          // the word and one centroid step to the residual's offset
+          const float kw = static_cast<float>(1u << (W * (pi % (GP / 2))));
+          const uint64_t kw2 = pk2(kw, kw);
+          const uint64_t y2 = pk2(__uint_as_float(yv[2 * i]), __uint_as_float(yv[2 * i + 1]));
+          uint64_t c2 = ncs02;
 #pragma unroll
           for (int t = 0; t < NL - 1; ++t) {
-            const bool gt = yv > T[t];
-            id += gt ? 1u : 0u;
-            c = gt ? cen[t + 1] : c;
+            const float2 th = up2(T2[t]);
+            const uint64_t ind = pk2(gt_one(__uint_as_float(yv[2 * i]), th.x),
+                                     gt_one(__uint_as_float(yv[2 * i + 1]), th.y));
+            c2 = fma2(ind, dcs2[t], c2);
+            if (pi < GP / 2) wa = fma2(ind, kw2, wa);
+            else wb = fma2(ind, kw2, wb);
           }
-          pk[(j * W) >> 5] |= id << ((j * W) & 31);
-          c2[e] = c;
+          const uint64_t r = fma2(y2, scl2, c2);
+          racc[pi & 3] = fma2(r, r, racc[pi & 3]);
+          // Veltkamp split: hi keeps the top 11 significant bits (exact in fp16 for |r| < 2^15),
+          // lo = r - hi exactly (13 bits, rounded to fp16's 11). c = RN(8193 r) comes from one
+          // fma so that no multiply is left for the compiler to fuse with the next subtraction.
+          const uint64_t cc = fma2(r, kSplit2, r);
+          const uint64_t hi = sub2(cc, sub2(cc, r));
+          const float2 hv = up2(hi), lv = up2(sub2(r, hi));
+          hw[pi] = h2_bits(hv.x, hv.y);
+          lw[pi] = h2_bits(lv.x, lv.y);
         }
-        const uint64_t r = fma2(mn2, pk2(c2[0], c2[1]), P[p]);
-        racc = fma2(r, r, racc);
-        const float2 v = up2(mul2(r, scl2));
-        const uint32_t hb = h2_bits(v.x, v.y);
-        const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hb));
-        const float2 lo = up2(sub2(pk2(v.x, v.y), pk2(hf.x, hf.y)));
-        hw[i] = hb;
-        lw[i] = h2_bits(lo.x, lo.y);
       }
-      tmem_st8(tlane + 128 + 8 * g, hw);
-      tmem_st8(tlane + 192 + 8 * g, lw);
-    }
-    const float2 r2 = up2(racc);
-    const __half r16 = __float2half_rn(sqrtf((r2.x + r2.y) * (1.f / 128.f)));
-    if (valid) {
-      const int64_t orow = out_row_tc(a.map, row);
-      uint4* dst = reinterpret_cast<uint4*>(a.idx + orow * IB);
+      if constexpr (GP == 8) {
+        tmem_st8(tlane + 128 + GP * g, *reinterpret_cast<uint32_t(*)[8]>(hw));
+        tmem_st8(tlane + 192 + GP * g, *reinterpret_cast<uint32_t(*)[8]>(lw));
+      } else {
 #pragma unroll
-      for (int w = 0; w < NW; w += 4) dst[w / 4] = make_uint4(pk[w], pk[w + 1], pk[w + 2], pk[w + 3]);
+        for (int q = 0; q < GP / 16; ++q) {
+          tmem_st16(tlane + 128 + GP * g + 16 * q, *reinterpret_cast<uint32_t(*)[16]>(hw + 16 * q));
+          tmem_st16(tlane + 192 + GP * g + 16 * q, *reinterpret_cast<uint32_t(*)[16]>(lw + 16 * q));
+        }
+      }
+      {
+        // exact integers below 2^16: adding 2^23 puts them in the low mantissa bits
+        const float2 fa = up2(add2(wa, pk2(8388608.f, 8388608.f)));
+        const float2 fb = up2(add2(wb, pk2(8388608.f, 8388608.f)));
+        constexpr int kHalfBits = W * GP / 2;
+        sCode[g * kTile + tid] = (__float_as_uint(fa.x) & 0xffffu) |
+                                 ((__float_as_uint(fb.x) & 0xffffu) << kHalfBits);
+        sCode[(NG + g) * kTile + tid] = (__float_as_uint(fa.y) & 0xffffu) |
+                                        ((__float_as_uint(fb.y) & 0xffffu) << kHalfBits);
+      }
+    }
+    const float2 r2 = up2(add2(add2(racc[0], racc[1]), add2(racc[2], racc[3])));
+    const float rss = r2.x + r2.y;
+    const __half r16 = __float2half_rn(sqrtf(rss * (1.f / 128.f)) / scl);
+    if (valid) {
+      const int64_t orow = out_row_tc(a.map, a.row_base + row);
+      uint4* dst = reinterpret_cast<uint4*>(a.idx + orow * (NW * 4));
+#pragma unroll
+      for (int w = 0; w < NW; w += 4)
+        dst[w / 4] = make_uint4(sCode[w * kTile + tid], sCode[(w + 1) * kTile + tid],
+                                sCode[(w + 2) * kTile + tid], sCode[(w + 3) * kTile + tid]);
       *reinterpret_cast<uint32_t*>(a.nrm + orow * 2) =
           static_cast<uint32_t>(half_bits(n16)) | (static_cast<uint32_t>(half_bits(r16)) << 16);
     }
     prev_row = row;
     prev_valid = valid;
+    prev_zero = !(rss > 0.f);
 
-    // ---- issue the MMAs of this tile; refill this staging buffer two tiles ahead
+    // ---- hand the tile to the tensor core; refill this staging buffer two tiles ahead
     tmem_st_wait();
     tc_fence_before();
-    __syncthreads();
+    mbar_arrive(&bar_a);
     if (tid == 0) {
+      if (ok) ok = mbar_wait_ns(&bar_a, static_cast<uint32_t>(k & 1), kWaitNs);
       tc_fence_after();
+      if (ok) {
 #pragma unroll
-      for (int s = 0; s < 16; ++s) {
-        const uint64_t bdesc = umma_desc(smem_u32(sB) + (s & 7) * 256, 128, 2048);
-        umma_f16_ts(tbase, tbase + 128 + 8 * s, bdesc, idesc, s > 0 ? 1u : 0u);
+        for (int s = 0; s < 16; ++s) {
+          const uint64_t bdesc = umma_desc(smem_u32(sB) + (s & 7) * 256, 128, 2048);
+          umma_f16_ts(tbase, tbase + 128 + 8 * s, bdesc, idesc, s > 0 ? 1u : 0u);
+        }
+        umma_commit(&bar_mma);
+        if (k + 2 < n_local) {
+          const int row0 = static_cast<int>((tile + 2 * grid) * kTile);
+          mbar_expect_tx(&bar_x[b], kXBuf);
+          tma_load_2d(sX + b * kXBuf, &tmap, 0, row0, &bar_x[b]);
+          tma_load_2d(sX + b * kXBuf + kXBuf / 2, &tmap, 64, row0, &bar_x[b]);
+        }
       }
-      umma_commit(&bar_mma);
     }
-    if (warp == 0 && k + 2 < n_local) issue_tile(a, sX + b * kXBuf, &bar_x[b], tile + 2 * grid, lane);
   }
 
-  if (!failed && n_local > 0) {
-    // sign bits of the last tile
-    if (__syncthreads_and(mbar_wait_ns(&bar_mma, static_cast<uint32_t>((n_local - 1) & 1), kWaitNs))) {
-      tc_fence_after();
-      store_signs(a, tlane, prev_valid, prev_row);
-    } else {
-      failed = true;
-    }
+  if (n_local > 0) {
+    if (ok) ok = mbar_wait_ns(&bar_mma, static_cast<uint32_t>((n_local - 1) & 1), kWaitNs);
+    tc_fence_after();
+    if (ok) store_signs(a, tlane, prev_valid, prev_zero, a.row_base + prev_row);
   }
-  if (failed) {
-    // a bounded wait gave up: report, let outstanding copies and MMAs land (bounded), leave
-    if (tid == 0) atomicOr(a.err, 1);
-    for (int bb = 0; bb < 2; ++bb) mbar_wait_ns(&bar_x[bb], 0, kWaitNs / 4);
-    mbar_wait_ns(&bar_mma, 0, kWaitNs / 4);
-  }
+  if (!ok) atomicOr(a.err, 1);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -335,8 +401,21 @@ __global__ void __launch_bounds__(128, 2) k_keys_prod_tc(const __grid_constant__
   }
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
 template <int MB>
-tq_status run_tc(const TcKeyArgs& a, cudaStream_t st) {
+tq_status run_tc(const CUtensorMap& tmap, const TcKeyArgs& a, cudaStream_t st) {
   auto kern = k_keys_prod_tc<MB>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -349,7 +428,7 @@ tq_status run_tc(const TcKeyArgs& a, cudaStream_t st) {
   cudaGetDevice(&dev);
   const int64_t cap = 2ll * sm_count(dev);
   const int grid = static_cast<int>(a.n_tiles < cap ? a.n_tiles : cap);
-  kern<<<grid, 128, kSmemBytes, st>>>(a);
+  kern<<<grid, 128, kSmemBytes, st>>>(tmap, a);
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ECUDA;
 }
 
@@ -358,7 +437,8 @@ tq_status run_tc(const TcKeyArgs& a, cudaStream_t st) {
 __device__ int g_tq_device_error = 0;
 
 bool keys_tc_ok(const tq_quantizer* q, int dtype) {
-  return q->mode == TQ_MODE_PROD && dtype == TQ_BF16 && q->bits >= 2 && q->bits <= 4;
+  return q->mode == TQ_MODE_PROD && dtype == TQ_BF16 && q->bits >= 2 && q->bits <= 4 &&
+         encode_fn() != nullptr;
 }
 
 tq_status launch_keys_tc(const tq_quantizer* q, const void* x, int64_t n_rows, int64_t ld,
@@ -367,14 +447,32 @@ tq_status launch_keys_tc(const tq_quantizer* q, const void* x, int64_t n_rows, i
   int* err = nullptr;
   if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_tq_device_error) != cudaSuccess)
     return TQ_ECUDA;
-  TcKeyArgs a{static_cast<const uint16_t*>(x), n_rows, ld, (n_rows + kTile - 1) / kTile,
-              q->dev, out.idx, out.signs, out.norms, map, err};
-  switch (q->bits) {
-    case 2: return run_tc<1>(a, st);
-    case 3: return run_tc<2>(a, st);
-    case 4: return run_tc<3>(a, st);
-    default: return TQ_EUNSUPPORTED;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (!enc) return TQ_ECUDA;
+  for (int64_t r0 = 0; r0 < n_rows; r0 += kChunkRows) {
+    const int64_t nr = n_rows - r0 < kChunkRows ? n_rows - r0 : kChunkRows;
+    // rows of 128 bf16 at a stride of ld elements; boxes of 64 columns x 128 rows
+    CUtensorMap tmap;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(nr)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+    const cuuint32_t box[2] = {64, kTile};
+    const cuuint32_t estr[2] = {1, 1};
+    void* base = const_cast<uint16_t*>(static_cast<const uint16_t*>(x) + r0 * ld);
+    if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return TQ_ECUDA;
+    TcKeyArgs a{nr, r0, (nr + kTile - 1) / kTile, q->dev, out.idx, out.signs, out.norms, map, err};
+    tq_status s;
+    switch (q->bits) {
+      case 2: s = run_tc<1>(tmap, a, st); break;
+      case 3: s = run_tc<2>(tmap, a, st); break;
+      case 4: s = run_tc<3>(tmap, a, st); break;
+      default: s = TQ_EUNSUPPORTED;
+    }
+    if (s != TQ_OK) return s;
   }
+  return TQ_OK;
 }
 
 tq_status take_device_error(cudaStream_t st) {

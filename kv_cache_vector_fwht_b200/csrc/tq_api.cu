@@ -150,7 +150,16 @@ tq_status tq_build_codebook(int d, int bits, int mode, uint64_t seed,
         std::memcpy(&h->s_rot[r * kD + c], &v, 2);
         std::memcpy(&h->s_rot_t[c * kD + r], &v, 2);
       }
+    for (int j = 0; j < kD; ++j)
+      for (int kk = 0; kk < kD; ++kk) {
+        const int col = (kk >> 1) + 64 * (kk & 1);
+        const size_t off = static_cast<size_t>(j >> 3) * 1024 + (kk >> 3) * 64 + (j & 7) * 8 + (kk & 7);
+        h->s_umma[off] = q->host.s_rot[j * kD + col];
+      }
   }
+  for (int qq = 0; qq < kD / 2; ++qq)
+    h->pair_mask[qq] = (q->host.signs[2 * qq] < 0 ? 1u << 15 : 0u) |
+                       (q->host.signs[2 * qq + 1] < 0 ? 1u << 31 : 0u);
   if (cudaGetDevice(&q->device) != cudaSuccess) {
     delete h;
     delete q;

@@ -28,6 +28,13 @@ struct DevTables {
   uint8_t chan[kD];        // grouped: outlier channels ascending, then normal channels ascending
   __half s_rot[kD * kD];   // prod: S_rot row-major (fp16-exact Gaussian)
   __half s_rot_t[kD * kD]; // prod: S_rot transposed (column j of S_rot contiguous)
+  // prod: S_rot as the tensor-core B operand image (fp16 bits): K order permuted so that
+  // k' = 2p holds column p and k' = 2p + 1 column p + 64, laid out in the canonical K-major
+  // no-swizzle form (element (j, k') at byte (j/8)*2048 + (k'/8)*128 + (j%8)*16 + (k'%8)*2).
+  alignas(16) uint16_t s_umma[kD * kD];
+  // rotation signs of bf16 element pairs: word q has bit 15 set if s_{2q} = -1, bit 31 if
+  // s_{2q+1} = -1 (an XOR flips both elements of a packed pair).
+  alignas(16) uint32_t pair_mask[kD / 2];
 };
 
 struct HostTables {
