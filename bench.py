@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--only", default="all", choices=["all", "decode", "quantize"],
                     help="run one leg only (small cases for profiling)")
     ap.add_argument("--quantize-rows", type=int, default=1 << 22, help="rows per layer")
+    ap.add_argument("--quantize-sweep", action="store_true",
+                    help="with --only quantize: every mode and width of the key-quantize sweep")
     return ap.parse_args()
 
 
@@ -161,6 +163,17 @@ def run_tq(args):
     dev = torch.device("cuda", local)
     peak, peak_kind = load_peaks()
     if args.only == "quantize":
+        if args.quantize_sweep:
+            out = {}
+            for mode, bits in [("mse", 1), ("mse", 2), ("mse", 3), ("mse", 4), ("prod", 2),
+                               ("prod", 3), ("prod", 4), ("grouped", 1), ("grouped", 2),
+                               ("grouped", 3)]:
+                out[f"{mode}{bits}"] = bench_quantize(tq, torch, dev, world, peak, peak_kind,
+                                                      rows=args.quantize_rows, mode=mode,
+                                                      bits=bits)
+            if rank == 0:
+                print(json.dumps({"key_quantize_sweep": out}))
+            return
         r = bench_quantize(tq, torch, dev, world, peak, peak_kind, rows=args.quantize_rows)
         if rank == 0:
             print(json.dumps({"key_quantize": r}))
@@ -287,9 +300,10 @@ def run_tq(args):
         dist.destroy_process_group()
 
 
-def bench_quantize(tq, torch, dev, world, peak, peak_kind, rows=1 << 22, reps=5):
-    """Key-quantize throughput: 4 layers x 2^22 bf16 rows (2^24 rows), 3-bit prod, quantizer
-    seed = layer, 32 channels at 4x std. Inputs (4 GiB) exceed L2; no flush needed."""
+def bench_quantize(tq, torch, dev, world, peak, peak_kind, rows=1 << 22, reps=5, mode="prod",
+                   bits=3):
+    """Key-quantize throughput: 4 layers x 2^22 bf16 rows (2^24 rows), 3-bit prod by default,
+    quantizer seed = layer, 32 channels at 4x std. Inputs (4 GiB) exceed L2; no flush needed."""
     import workloads as W
     ch = torch.from_numpy(W.outlier_channels(4)).long().to(dev)
     g = torch.Generator(device=dev).manual_seed(4)
@@ -299,7 +313,8 @@ def bench_quantize(tq, torch, dev, world, peak, peak_kind, rows=1 << 22, reps=5)
         x[:, ch] *= 4.0
         xs.append(x.to(torch.bfloat16))
         del x
-        qs.append(tq.tq_build_codebook(128, 3, "prod", layer))
+        qs.append(tq.tq_build_codebook(128, bits, mode, layer,
+                                       W.outlier_channels(4) if mode == "grouped" else None))
         planes.append(qs[-1].alloc_key_planes(rows, dev))
     st = torch.cuda.current_stream()
     for layer in range(4):
@@ -317,12 +332,18 @@ def bench_quantize(tq, torch, dev, world, peak, peak_kind, rows=1 << 22, reps=5)
     tq.tq_sync_status()
     ms = sum(times) / len(times)
     n = 4 * rows
-    gbs = n * (256 + KEY_BYTES) / (ms / 1e3) / 1e9
+    lay = qs[0].layout
+    out_bytes = lay["idx_bytes"] + lay["sign_bytes"] + 2 * lay["n_norms"]
+    gbs = n * (256 + out_bytes) / (ms / 1e3) / 1e9
+    kernel = {"prod": f"k_keys_prod_tc<{bits - 1}>", "mse": f"k_keys_full<mse,{bits}>",
+              "grouped": f"k_keys_grouped<{bits}>"}[mode]
+    del xs, planes
+    torch.cuda.empty_cache()
     return {"rows_per_s": n / (ms / 1e3), "ms_per_pass": ms, "rows_per_pass": n,
-            "mode": "prod b=3",
+            "mode": f"{mode} b={bits}",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                          "frac": gbs / peak, "traffic": None,
-                         "bytes_per_row": 256 + KEY_BYTES, "kernel": "k_keys_prod_tc<2>",
+                         "bytes_per_row": 256 + out_bytes, "kernel": kernel,
                          "peak_kind": f"{peak_kind} (hbm_gbs, burst)"}}
 
 

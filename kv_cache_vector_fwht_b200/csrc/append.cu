@@ -43,6 +43,9 @@ __global__ void __launch_bounds__(256) k_append(const __grid_constant__ AppendAr
   __shared__ __align__(16) uint8_t sB[PROD ? 2 * kRowsPerCta * kSStride : 16];
   __shared__ float sD[PROD ? kD * (kRowsPerCta + 1) : 1];
 
+  // a decode launched next may start its query-only prologue now (it waits for this grid
+  // before it reads the lengths or the cache)
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const DevTables* __restrict__ tab = a.tab;
   if constexpr (PROD) {

@@ -4,26 +4,29 @@
 // attention_score):  s_i = n16_i <Pi q, c[idx_i]> + r16_i sqrt(pi/2)/d <S q, 2 sigma_i - 1>.
 // With q_rot = H (s . q) (so Pi q = q_rot / sqrt(d)) and Sq = S_rot q_rot / sqrt(d):
 //   <Pi q, c[idx]> = (1/d) sum_j q_rot_j C[idx_j]      (C: N(0,1)-scale centroids).
-// Both sums are read from per-query lookup tables in shared memory; the kernel consumes the
-// packed bytes directly (TurboQuant bit-packing article, section 5).
+// Both sums are read from per-query byte lookup tables in shared memory; the kernel consumes
+// the packed bytes directly (TurboQuant bit-packing article, section 5).
 //
-// Lookup tables. A field is the packed bits covering consecutive coordinates: a 2-bit index
-// byte (4 coordinates), a byte of two 3-bit indices in nibbles (2 coordinates), a 1-bit index
-// nibble (4 coordinates) or a QJL sign nibble (4 coordinates). The Lloyd-Max codebook is
-// symmetric (C[L-1-k] = -C[k]) and the sign sums are odd, so the value of a field and of its
-// mirror (all codes k -> L-1-k, all signs flipped) differ only in sign: a table keeps the
-// canonical half of the fields (top code bit clear) and a lookup returns (entry, +-1).
-// Entries hold 4 query heads (16 bytes); 8 heads use two such tables. Entry e of position p
-// sits at ((e * P + p) * 16) bytes, so position p lives in bank group p mod 8 and the eight
-// lanes of one 16-byte shared-memory phase (walking positions p = lane + s) never collide.
-// Tables are pre-multiplied by sm_scale * log2(e): the online softmax runs in base 2.
+// Byte tables. Every packed byte is one lookup: a 2-bit index byte covers 4 coordinates, a
+// 1-bit index byte 8, a byte of two 3-bit indices (in nibbles) 2, a QJL sign byte 8. The
+// Lloyd-Max codebook is symmetric (C[L-1-k] = -C[k]) and the sign sums are odd, so the value
+// of a byte and of its mirror (every code k -> L-1-k, every sign flipped) differ only in sign:
+// a table keeps the canonical half (top bit clear) and a lookup returns (entry, +-1). An
+// entry holds 4 query heads (16 bytes); a CTA serves at most 4 heads. Entry e of position p
+// sits at (e * P + p) * 16 bytes. At step i of an 8-position block, lane l reads position
+// 8 b + ((l + i) mod 8), so the eight lanes of one 16-byte shared-memory phase fall in eight
+// different bank groups. Tables are pre-multiplied by sm_scale * log2(e): the online softmax
+// runs in base 2.
 //
-// Grid: (context split, head group, sequence). A CTA takes one KV head, up to 8 of its query
-// heads and a contiguous token range; it streams packed K/V tiles of 256 tokens through a
-// cp.async double buffer; lane l of warp w scores token 32w + l; then lanes split the 128
-// channels of P.V (8 per lane, two tokens per step) with packed fp32x2 FMAs. Each CTA merges
-// its warps and writes a partial (m, l, o); the last CTA of a (sequence, head group) to
-// finish merges all partials (an atomic counter, no waiting).
+// Grid: (context split, head group, sequence); a CTA takes one KV head, up to 4 of its query
+// heads and a contiguous token range, with 16 warps. Warp w walks its own 32-token chunks
+// (chunk w, w + 16, ... of the range), so no CTA-wide barrier sits in the loop: each lane
+// holds its token's key bytes in registers (prefetched one chunk ahead), scores it from the
+// tables, and the warp runs the online softmax; the chunk's value bytes arrive in the warp's
+// own shared-memory slot by cp.async, and for P.V the lanes split the 128 channels (4 per
+// lane, one token a step) with packed fp32x2 FMAs. Each CTA merges its warps and writes a
+// partial (m, l, o); the last CTA of a (sequence, head group) to finish merges all partials
+// (an atomic counter, no waiting).
 #include <cfloat>
 #include <cmath>
 #include <mutex>
@@ -34,12 +37,16 @@
 namespace tq {
 namespace {
 
-constexpr int kMaxHeads = 8;      // query heads per CTA
-constexpr int kMaxGroups = 128;
-constexpr int kTile = 256;        // tokens per tile (8 warps x 32)
-constexpr int kThreads = 256;
+constexpr int kMaxHeads = 4;      // query heads per CTA (one 16-byte table entry)
+constexpr int kMaxGroups = 256;
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kChunkStride = 32 * kWarps;  // tokens between a warp's consecutive chunks
 constexpr int kPartStride = 132;  // floats per (head, split) partial: m, l, pad, o[128]
-constexpr int kSrotStride = 272;  // bytes per staged S_rot row (256 + 16: bank spread)
+constexpr int kSrotStride = 272;  // bytes per staged q half row (256 + 16: bank spread)
+// dequant pairs of a warp: [group][token] float4 rows of 34 entries, so that the 4 groups x 2
+// tokens read by one P.V step fall in 8 different 16-byte bank groups
+constexpr int kVpStride = 34;
 
 struct DecodeArgs {
   const uint8_t* k_idx;
@@ -58,11 +65,18 @@ struct DecodeArgs {
   int n_kv_heads, capacity, n_q_heads;
   int q_f32, out_f32;
   int n_splits, tokens_per_split;
+  int max_len;  // host copy of the longest sequence (an upper bound of every len[b])
   float scale_log2, inv_scale_log2;
   int16_t g_kv[kMaxGroups];
   int16_t g_heads[kMaxGroups][kMaxHeads];
   int8_t g_n[kMaxGroups];
 };
+
+// Programmatic dependent launch: wait until the grids this one depends on have completed and
+// their memory is visible (a no-op when the kernel was launched without the attribute).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
 
 // (+1.0, +1.0) or (-1.0, -1.0) from an all-ones / all-zeros mask
 __device__ __forceinline__ uint64_t sign_pair(int mask) {
@@ -70,110 +84,87 @@ __device__ __forceinline__ uint64_t sign_pair(int mask) {
   return pk2(s, s);
 }
 
-// Shared-memory plan. A table has P positions of E canonical 16-byte entries (4 heads);
-// positions are stored P + 32 times wide where noted (entry p + P repeats entry p) so that
-// lane l's walk p = l + s never wraps and s becomes an immediate load offset.
-template <int MB, int VB, int NH4>
+// Shared-memory plan.
+template <int MB, int VB>
 struct Lay {
-  static constexpr int IB = kD * storage_width_c(MB) / 8;            // index bytes per token
-  static constexpr bool NIB = MB != 3;                               // nibble index tables
-  static constexpr int PI = MB == 2 ? 64 : (MB == 1 ? 32 : 64);      // index positions
-  static constexpr int EI = MB == 3 ? 32 : 8;                        // canonical entries
-  static constexpr int PDI = NIB ? PI + 32 : PI;                     // stored positions
-  static constexpr int HALF_I = EI * PDI * 16;
-  static constexpr int PDS = 64;                                     // sign table, stored
-  static constexpr int HALF_S = 8 * PDS * 16;
-  static constexpr int STAGES = MB == 3 ? 2 : 1;
-  static constexpr int VQB = VB ? kD * VB / 8 : 0;
-  static constexpr int VPB = VB ? 16 : 0;
-  // one tile stage
-  static constexpr int o_idx = 0;
-  static constexpr int o_sgn = o_idx + kTile * IB;
-  static constexpr int o_nrm = o_sgn + kTile * 16;
-  static constexpr int o_vq = o_nrm + kTile * 4;
-  static constexpr int o_vp = o_vq + kTile * VQB;
-  static constexpr int stage = o_vp + kTile * VPB;
-  // regions: tables, query buffers,
-  // tile stages, then per-warp p pairs and dequant pairs (tiles..end reused for the merge)
-  static constexpr int lut_bytes = NH4 * (HALF_I + HALF_S);
+  static constexpr int IB = kD * storage_width_c(MB) / 8;  // index bytes per token
+  static constexpr int PI = IB;                            // index positions (bytes)
+  static constexpr int EI = MB == 3 ? 32 : 128;            // canonical entries per position
+  static constexpr int PS = 16;                            // sign positions
+  static constexpr int ES = 128;
+  static constexpr int VQB = VB ? kD * VB / 8 : 0;         // value code bytes per token
+  static constexpr int VPB = VB ? 16 : 0;                  // value params per token
   static constexpr int lutI = 0;
-  static constexpr int lutS = NH4 * HALF_I;
-  static constexpr int qrT = (lut_bytes + 127) & ~127;               // q_rot [128][8] f32
-  static constexpr int sqT = qrT + kD * kMaxHeads * 4;               // Sq    [128][8] f32
+  static constexpr int lutS = lutI + EI * PI * 16;
+  static constexpr int qrT = lutS + ES * PS * 16;                    // q_rot [128][4] f32
+  static constexpr int sqT = qrT + kD * kMaxHeads * 4;               // Sq    [128][4] f32
   static constexpr int qhi = sqT + kD * kMaxHeads * 4;               // hi [8][136] f16
-  static constexpr int qlo = qhi + kMaxHeads * kSrotStride;          // lo [8][136] f16
-  static constexpr int qinv = qlo + kMaxHeads * kSrotStride;         // [8] f32
-  static constexpr int tiles = (qinv + 32 + 127) & ~127;
-  static constexpr int ppair = tiles + STAGES * stage;               // [8][32][8] (p, p)
-  static constexpr int vpair = ppair + 8 * 32 * kMaxHeads * 8;       // [8][32][4] (s16,s16,c,c)
-  static constexpr int end_v = vpair + (VB ? 8 * 32 * 4 * 16 : 0);
-  static constexpr int merge = 8 * kMaxHeads * kPartStride * 4;
-  static constexpr int total = (end_v - tiles) >= merge ? end_v : tiles + merge;
+  static constexpr int qlo = qhi + 8 * kSrotStride;                  // lo [8][136] f16
+  static constexpr int qinv = qlo + 8 * kSrotStride;                 // [8] f32
+  // per-warp slots: value bytes of the chunk, p pairs, dequant pairs
+  static constexpr int wv = (qinv + 32 + 127) & ~127;
+  static constexpr int wv_bytes = 32 * (VQB + VPB);
+  static constexpr int o_vq = 0;                 // within a warp's value slot
+  static constexpr int o_vp = 32 * VQB;
+  static_assert(o_vq == 0 && o_vp >= 0, "value slot layout");
+  static constexpr int ppair = wv + kWarps * wv_bytes;                 // [warp][2][32] 2x(p, p)
+  static constexpr int vpair = ppair + kWarps * 32 * kMaxHeads * 8;    // [warp][4][34] f32x4
+  static constexpr int end_v = vpair + (VB ? kWarps * 4 * kVpStride * 16 : 0);
+  static constexpr int merge = kWarps * kMaxHeads * kPartStride * 4;   // reuses wv..
+  // prologue scratch for the nibble partial tables (the value slots may be filling then)
+  static constexpr int scratch = VB ? ppair : wv;
+  static constexpr int scratch_bytes = (2 * 16 * (MB == 3 ? 0 : PI) + 2 * 16 * PS) * 16;
+  static constexpr int total = (end_v - wv) >= merge ? end_v : wv + merge;
+  static_assert(scratch + scratch_bytes <= total, "prologue scratch fits");
 };
 
-template <int MB, int VB, int NH4>
-__device__ __forceinline__ void load_tile(uint8_t* st, const DecodeArgs& a, int64_t rowbase,
-                                          int n) {
-  using Lo = Lay<MB, VB, NH4>;
-  // n: tokens to copy (a multiple of 4, within capacity)
-  const int c_idx = n * Lo::IB / 16, c_sgn = n, c_nrm = n / 4;
-  const int c_vq = n * Lo::VQB / 16, c_vp = VB ? n : 0;
-  const int total = c_idx + c_sgn + c_nrm + c_vq + c_vp;
-  for (int c = threadIdx.x; c < total; c += kThreads) {
-    int r = c;
-    const uint8_t* src;
-    uint8_t* dst;
-    if (r < c_idx) {
-      src = a.k_idx + rowbase * Lo::IB + 16 * r;
-      dst = st + Lo::o_idx + 16 * r;
-    } else if ((r -= c_idx) < c_sgn) {
-      src = a.k_sgn + rowbase * 16 + 16 * r;
-      dst = st + Lo::o_sgn + 16 * r;
-    } else if ((r -= c_sgn) < c_nrm) {
-      src = reinterpret_cast<const uint8_t*>(a.k_nrm) + rowbase * 4 + 16 * r;
-      dst = st + Lo::o_nrm + 16 * r;
-    } else if ((r -= c_nrm) < c_vq) {
-      src = a.v_q + rowbase * Lo::VQB + 16 * r;
-      dst = st + Lo::o_vq + 16 * r;
-    } else {
-      r -= c_vq;
-      src = reinterpret_cast<const uint8_t*>(a.v_par) + rowbase * 16 + 16 * r;
-      dst = st + Lo::o_vp + 16 * r;
-    }
-    cp_async16(dst, src, true);
-  }
-}
-
-// Accumulate one 4-head (or 8-head) table entry with sign: acc[j] += sg * entry.
-template <int NH4, int HALF>
-__device__ __forceinline__ void lut_acc(uint64_t (&acc)[4], const uint8_t* p, uint64_t sg) {
+// Accumulate one 4-head table entry with sign: acc[j] += sg * entry.
+__device__ __forceinline__ void lut_acc(uint64_t (&acc)[2], const uint8_t* p, uint64_t sg) {
   const ulonglong2 L = *reinterpret_cast<const ulonglong2*>(p);
   acc[0] = fma2(sg, L.x, acc[0]);
   acc[1] = fma2(sg, L.y, acc[1]);
-  if constexpr (NH4 == 2) {
-    const ulonglong2 M = *reinterpret_cast<const ulonglong2*>(p + HALF);
-    acc[2] = fma2(sg, M.x, acc[2]);
-    acc[3] = fma2(sg, M.y, acc[3]);
+}
+
+// Byte k of w sign-extended to 32 bits (prmt: a selector nibble with its top bit set
+// replicates the selected byte's sign bit).
+__device__ __forceinline__ int byte_sx(uint32_t w, int k) {
+  const uint32_t sel = static_cast<uint32_t>(k) | ((8u | k) << 4) | ((8u | k) << 8) | ((8u | k) << 12);
+  uint32_t d;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(d) : "r"(w), "r"(sel));
+  return static_cast<int>(d);
+}
+
+// The 8-byte block (w0, w1) rotated right by this lane's r = l mod 8 bytes: byte i of
+// (out0, out1) is byte (r + i) mod 8 of the block.
+__device__ __forceinline__ void rot_block(uint32_t w0, uint32_t w1, bool swap, uint32_t sh,
+                                          uint32_t& out0, uint32_t& out1) {
+  const uint32_t a = swap ? w1 : w0, b = swap ? w0 : w1;
+  out0 = __funnelshift_r(a, b, sh);
+  out1 = __funnelshift_r(b, a, sh);
+}
+
+// Lookups of one 8-byte block of mirror-symmetric bytes (index bytes of 1- or 2-bit codes,
+// or sign bytes): byte i of the rotated block is position 8 blk + ((l + i) mod 8).
+template <int ROWB>
+__device__ __forceinline__ void block_lookups(uint64_t (&acc)[2], uint32_t R0, uint32_t R1,
+                                              const uint8_t* tab, int blk,
+                                              const uint32_t (&rot16)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t R = i < 4 ? R0 : R1;
+    const int sx = byte_sx(R, i & 3);
+    const int msk = sx >> 31;
+    const uint32_t e = static_cast<uint32_t>(sx ^ msk);  // canonical entry, 0..127
+    const uint8_t* p = tab + 128 * blk + e * ROWB + rot16[i];
+    lut_acc(acc, p, sign_pair(msk));
   }
 }
 
-// Nibble-table lookup for nibble s of the lane-rotated words R (field sign-extended from its
-// top bit: negative fields use the mirrored canonical entry with sign -1).
-template <int NH4, int HALF, int STRIDE>
-__device__ __forceinline__ void nib_step(uint64_t (&acc)[4], uint32_t w, int k, const uint8_t* lane_base,
-                                         int s) {
-  const int t = static_cast<int>(w << (28 - 4 * k)) >> 28;
-  const int msk = t >> 31;
-  const uint8_t* p = lane_base + (t ^ msk) * STRIDE + 16 * s;
-  lut_acc<NH4, HALF>(acc, p, sign_pair(msk));
-}
-
-template <int MB, int VB, int NH4>
-__global__ void __launch_bounds__(kThreads, MB == 3 ? 1 : 2)
-k_decode(const __grid_constant__ DecodeArgs a) {
-  using Lo = Lay<MB, VB, NH4>;
-  constexpr int IB = Lo::IB, PI = Lo::PI, EI = Lo::EI, PDI = Lo::PDI;
-  constexpr int NH = 4 * NH4;
+template <int MB, int VB, int NH>
+__global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ DecodeArgs a) {
+  using Lo = Lay<MB, VB>;
+  constexpr int IB = Lo::IB, PI = Lo::PI;
+  static_assert(NH >= 1 && NH <= kMaxHeads, "heads per CTA");
   constexpr bool HAS_V = VB != 0;
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* lutI = smem + Lo::lutI;
@@ -183,42 +174,88 @@ k_decode(const __grid_constant__ DecodeArgs a) {
   uint8_t* qhi = smem + Lo::qhi;
   uint8_t* qlo = smem + Lo::qlo;
   float* qinv = reinterpret_cast<float*>(smem + Lo::qinv);
-  uint8_t* tiles = smem + Lo::tiles;
   __shared__ int sLast;
   __shared__ float sCen[16];
 
   const int split = blockIdx.x, grp = blockIdx.y, b = blockIdx.z;
   const int kv = a.g_kv[grp], nh = a.g_n[grp];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int L = a.len[b];
   const int t0 = split * a.tokens_per_split;
-  const int t1 = min(L, t0 + a.tokens_per_split);
   const int64_t kvrow = (static_cast<int64_t>(b) * a.n_kv_heads + kv) * a.capacity;
 
+  // P.V: half-warp hw = lane / 16 takes every other token of a chunk; lane owns channels
+  // 8 j16 .. 8 j16 + 7 (j16 = lane mod 16) as four fp32 pairs
   float m[NH], l[NH];
-  uint64_t o[NH][2];   // channels (4 lane, 4 lane + 1), (4 lane + 2, 4 lane + 3)
+  uint64_t o[NH][4];
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
     m[h] = -INFINITY;
     l[h] = 0.f;
-    o[h][0] = 0ull;
-    o[h][1] = 0ull;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) o[h][k] = 0ull;
   }
 
-  if (t0 < t1) {
-    auto tile_count = [&](int ts) {
-      const int want = min(kTile, t1 - ts);
-      const int n4 = (want + 3) & ~3;
-      return min(n4, a.capacity - ts);
-    };
-    load_tile<MB, VB, NH4>(tiles, a, kvrow + t0, tile_count(t0));
-    cp_async_commit();
-
-    // ---------------- prologue (b1): rotate q, project with S_rot, build the tables
-    const DevTables* __restrict__ tab = a.tab;
-    // this warp's S_rot rows [16 warp, 16 warp + 16) as mma.sync A fragments, read from L2
-    uint32_t afr[8][4];
+  // The prologue reads only the query and the quantizer's tables, so it runs before the
+  // grid-dependency wait: launched after tq_append, it overlaps the append kernel (which
+  // signals its dependents at entry). The lengths and the cache are read after the wait.
+  int t1 = t0;
+  if (t0 < a.max_len) {
+    // warm L2 with this CTA's packed rows (all of them lie below the capacity); the reads
+    // proper come after the dependency wait (L2 is the point of coherence for the append)
     {
+      const int tp1 = min(a.max_len, t0 + a.tokens_per_split);
+      const int n = tp1 - t0;
+      const uint8_t* rng[5] = {a.k_idx + (kvrow + t0) * Lay<MB, VB>::IB, a.k_sgn + (kvrow + t0) * 16,
+                               reinterpret_cast<const uint8_t*>(a.k_nrm) + (kvrow + t0) * 4,
+                               a.v_q + (kvrow + t0) * Lay<MB, VB>::VQB,
+                               reinterpret_cast<const uint8_t*>(a.v_par) + (kvrow + t0) * 16};
+      const int len_b[5] = {n * Lay<MB, VB>::IB, n * 16, n * 4, n * Lay<MB, VB>::VQB, VB ? n * 16 : 0};
+#pragma unroll
+      for (int r = 0; r < 5; ++r)
+        for (int off = threadIdx.x * 128; off < len_b[r]; off += kThreads * 128)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(rng[r] + off));
+    }
+    // key bytes of this lane's token in chunk c (zeros past the range)
+    uint32_t kw[IB / 4], sw4[4], nw;
+    auto load_keys = [&](int ts, uint32_t (&iw)[IB / 4], uint32_t (&sg)[4], uint32_t& nn) {
+      const int t = ts + lane;
+      if (t < t1) {
+        const uint4* ip = reinterpret_cast<const uint4*>(a.k_idx + (kvrow + t) * IB);
+#pragma unroll
+        for (int i = 0; i < IB / 16; ++i) {
+          const uint4 v = __ldg(ip + i);
+          iw[4 * i] = v.x; iw[4 * i + 1] = v.y; iw[4 * i + 2] = v.z; iw[4 * i + 3] = v.w;
+        }
+        const uint4 s4 = __ldg(reinterpret_cast<const uint4*>(a.k_sgn + (kvrow + t) * 16));
+        sg[0] = s4.x; sg[1] = s4.y; sg[2] = s4.z; sg[3] = s4.w;
+        nn = __ldg(reinterpret_cast<const uint32_t*>(a.k_nrm) + kvrow + t);
+      } else {
+#pragma unroll
+        for (int i = 0; i < IB / 4; ++i) iw[i] = 0u;
+        sg[0] = sg[1] = sg[2] = sg[3] = 0u;
+        nn = 0u;
+      }
+    };
+    // value bytes of chunk ts into this warp's slot (cp.async, 16-byte pieces)
+    uint8_t* wslot = smem + Lo::wv + warp * Lo::wv_bytes;
+    auto load_values = [&](int ts) {
+      if constexpr (HAS_V) {
+        const int n = min(32, t1 - ts);  // tokens of the chunk (>= 1)
+        const int cq = n * Lo::VQB / 16, cp = n;
+        for (int c = lane; c < cq + cp; c += 32) {
+          if (c < cq) cp_async16(wslot + Lo::o_vq + 16 * c, a.v_q + (kvrow + ts) * Lo::VQB + 16 * c, true);
+          else cp_async16(wslot + Lo::o_vp + 16 * (c - cq),
+                          reinterpret_cast<const uint8_t*>(a.v_par) + (kvrow + ts + (c - cq)) * 16, true);
+        }
+      }
+      cp_async_commit();
+    };
+
+    // ---------------- prologue: rotate q, project with S_rot, build the tables
+    const DevTables* __restrict__ tab = a.tab;
+    // S_rot rows [16 warp, 16 warp + 16) as mma.sync A fragments (warps 0..7), from L2
+    uint32_t afr[8][4];
+    if (warp < 8) {
       const int g = lane >> 2, t = lane & 3;
       const uint32_t* r0 = reinterpret_cast<const uint32_t*>(tab->s_rot + (16 * warp + g) * kD);
       const uint32_t* r1 = r0 + 8 * kD / 2;
@@ -230,9 +267,9 @@ k_decode(const __grid_constant__ DecodeArgs a) {
         afr[kk][3] = __ldg(r1 + kk * 8 + 4 + t);
       }
     }
-    {
-      // q_rot of head `warp` (zeros for padded heads): signs, then the 128-point transform
-      // with 4 values per lane (2 stages in registers, 5 across lanes)
+    if (warp < 8) {
+      // q_rot of head slot `warp` (zeros for empty slots): signs, then the 128-point
+      // transform with 4 values per lane (2 stages in registers, 5 across lanes)
       float v[4] = {0.f, 0.f, 0.f, 0.f};
       if (warp < nh) {
         const int hq = a.g_heads[grp][warp];
@@ -263,7 +300,7 @@ k_decode(const __grid_constant__ DecodeArgs a) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int j = 4 * lane + i;
-        qrT[j * kMaxHeads + warp] = v[i];
+        if (warp < kMaxHeads) qrT[j * kMaxHeads + warp] = v[i];
         const float sv = v[i] * scl;
         const __half hi = __float2half_rn(sv);
         const __half lo = __float2half_rn(sv - __half2float(hi));
@@ -273,8 +310,8 @@ k_decode(const __grid_constant__ DecodeArgs a) {
     }
     if (threadIdx.x < 16) sCen[threadIdx.x] = tab->cent[0][threadIdx.x];
     __syncthreads();
-    {
-      // Sq = S_rot q_rot / sqrt(d) for the 8 head slots on tensor cores: mma.sync m16n8k16
+    if (warp < 8) {
+      // Sq = S_rot q_rot / sqrt(d) for the head slots on tensor cores: mma.sync m16n8k16
       // (fp16 S_rot is exact; q_rot enters as hi + lo fp16 halves; fp32 accumulation).
       const int g = lane >> 2, t = lane & 3;
       float c0 = 0.f, c1 = 0.f, c2 = 0.f, c3 = 0.f;
@@ -293,259 +330,269 @@ k_decode(const __grid_constant__ DecodeArgs a) {
               : "r"(afr[kk][0]), "r"(afr[kk][1]), "r"(afr[kk][2]), "r"(afr[kk][3]), "r"(b0), "r"(b1));
         }
       }
-      const float s0 = qinv[2 * t] * 0.088388347648318440550f;      // / sqrt(128)
-      const float s1 = qinv[2 * t + 1] * 0.088388347648318440550f;
-      const int j0 = 16 * warp + g;
-      sqT[j0 * kMaxHeads + 2 * t] = c0 * s0;
-      sqT[j0 * kMaxHeads + 2 * t + 1] = c1 * s1;
-      sqT[(j0 + 8) * kMaxHeads + 2 * t] = c2 * s0;
-      sqT[(j0 + 8) * kMaxHeads + 2 * t + 1] = c3 * s1;
+      if (2 * t < kMaxHeads) {  // columns 2t, 2t + 1 are head slots 0..3
+        const float s0 = qinv[2 * t] * 0.088388347648318440550f;      // / sqrt(128)
+        const float s1 = qinv[2 * t + 1] * 0.088388347648318440550f;
+        const int j0 = 16 * warp + g;
+        sqT[j0 * kMaxHeads + 2 * t] = c0 * s0;
+        sqT[j0 * kMaxHeads + 2 * t + 1] = c1 * s1;
+        sqT[(j0 + 8) * kMaxHeads + 2 * t] = c2 * s0;
+        sqT[(j0 + 8) * kMaxHeads + 2 * t + 1] = c3 * s1;
+      }
     }
     __syncthreads();
+    grid_dependency_wait();
+    t1 = min(a.len[b], t0 + a.tokens_per_split);
+    const int c0 = t0 + 32 * warp;
+    if (c0 < t1) {
+      load_keys(c0, kw, sw4, nw);
+      load_values(c0);
+    }
     {
       const float* cen = sCen;
       const float cI = a.scale_log2 * (1.f / 128.f);
       const float cS = a.scale_log2 * 1.2533141373155002512f / 128.f;  // sqrt(pi/2) / d
-      // index tables: one thread per (4-head half, stored position), all entries of it
-      for (int e = threadIdx.x; e < NH4 * PDI; e += kThreads) {
-        const int hf = e / PDI, pd = e - hf * PDI;
-        const int p = pd < PI ? pd : pd - PI;
-        uint8_t* dst = lutI + hf * Lo::HALF_I + pd * 16;
-        if constexpr (MB == 1) {          // nibble: four 1-bit codes (C = -c, +c), coords 4p..4p+3
-          const float c = cen[1] * cI;
-          float4 x[4];
+      // Byte entries are sums of two nibble partials (low and high half of the byte):
+      // NI[half][n][p] and NS[half][n][p] (16-byte float4 of the 4 head slots) are built in a
+      // scratch region first; entry (e, p) = N[0][e mod 16][p] + N[1][e / 16][p].
+      float4* NI = reinterpret_cast<float4*>(smem + Lo::scratch);
+      float4* NS = NI + (MB == 3 ? 0 : 2 * 16 * PI);
+      constexpr int PN = MB == 2 ? PI : (MB == 1 ? PI : 0);  // nibble positions = byte positions
+      if constexpr (MB != 3) {
+        constexpr int CPN = MB == 2 ? 2 : 4;  // coordinates per nibble
+        for (int i = threadIdx.x; i < 2 * 16 * PN; i += kThreads) {
+          const int pp = i % PN, n = (i / PN) % 16, hf = i / (16 * PN);
+          float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-          for (int f = 0; f < 4; ++f) x[f] = *reinterpret_cast<const float4*>(qrT + (4 * p + f) * kMaxHeads + 4 * hf);
-#pragma unroll
-          for (int en = 0; en < 8; ++en) {
-            float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int f = 0; f < 4; ++f) {
-              const float sg = ((en >> f) & 1) ? c : -c;
-              r.x = fmaf(x[f].x, sg, r.x); r.y = fmaf(x[f].y, sg, r.y);
-              r.z = fmaf(x[f].z, sg, r.z); r.w = fmaf(x[f].w, sg, r.w);
-            }
-            *reinterpret_cast<float4*>(dst + en * PDI * 16) = r;
+          for (int f = 0; f < CPN; ++f) {
+            const float4 x = *reinterpret_cast<const float4*>(qrT + (2 * CPN * pp + CPN * hf + f) * kMaxHeads);
+            const float c = cen[(n >> (MB * f)) & ((1 << MB) - 1)] * cI;
+            r.x = fmaf(x.x, c, r.x); r.y = fmaf(x.y, c, r.y);
+            r.z = fmaf(x.z, c, r.z); r.w = fmaf(x.w, c, r.w);
           }
-        } else {                          // two codes (2-bit nibble or 3-bit byte), coords 2p, 2p+1
-          const float4 x = *reinterpret_cast<const float4*>(qrT + (2 * p) * kMaxHeads + 4 * hf);
-          const float4 y = *reinterpret_cast<const float4*>(qrT + (2 * p + 1) * kMaxHeads + 4 * hf);
-          constexpr int LO = MB == 2 ? 4 : 8;     // levels of the first code
-#pragma unroll
-          for (int en = 0; en < EI; ++en) {
-            const float c0 = cen[en % LO] * cI, c1 = cen[en / LO] * cI;
-            *reinterpret_cast<float4*>(dst + en * PDI * 16) =
-                make_float4(fmaf(x.x, c0, y.x * c1), fmaf(x.y, c0, y.y * c1),
-                            fmaf(x.z, c0, y.z * c1), fmaf(x.w, c0, y.w * c1));
-          }
+          NI[(hf * 16 + n) * PN + pp] = r;
         }
       }
-      // QJL sign tables: entry bit f = sign bit of coordinate 4p + f (+1 if set, else -1)
-      for (int e = threadIdx.x; e < NH4 * Lo::PDS; e += kThreads) {
-        const int hf = e / Lo::PDS, pd = e - hf * Lo::PDS, p = pd & 31;
-        float4 x[4];
+      for (int i = threadIdx.x; i < 2 * 16 * Lo::PS; i += kThreads) {
+        const int pp = i % Lo::PS, n = (i / Lo::PS) % 16, hf = i / (16 * Lo::PS);
+        float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int f = 0; f < 4; ++f) x[f] = *reinterpret_cast<const float4*>(sqT + (4 * p + f) * kMaxHeads + 4 * hf);
-        uint8_t* dst = lutS + hf * Lo::HALF_S + pd * 16;
-#pragma unroll
-        for (int en = 0; en < 8; ++en) {
-          float4 r = make_float4(-x[3].x * cS, -x[3].y * cS, -x[3].z * cS, -x[3].w * cS);
-#pragma unroll
-          for (int f = 0; f < 3; ++f) {
-            const float sg = ((en >> f) & 1) ? cS : -cS;
-            r.x = fmaf(x[f].x, sg, r.x); r.y = fmaf(x[f].y, sg, r.y);
-            r.z = fmaf(x[f].z, sg, r.z); r.w = fmaf(x[f].w, sg, r.w);
-          }
-          *reinterpret_cast<float4*>(dst + en * Lo::PDS * 16) = r;
+        for (int f = 0; f < 4; ++f) {
+          const float4 x = *reinterpret_cast<const float4*>(sqT + (8 * pp + 4 * hf + f) * kMaxHeads);
+          const float sg = ((n >> f) & 1) ? cS : -cS;
+          r.x = fmaf(x.x, sg, r.x); r.y = fmaf(x.y, sg, r.y);
+          r.z = fmaf(x.z, sg, r.z); r.w = fmaf(x.w, sg, r.w);
         }
+        NS[(hf * 16 + n) * Lo::PS + pp] = r;
+      }
+      __syncthreads();
+      if constexpr (MB == 3) {
+        // byte = two 3-bit codes in nibbles: coords 2p, 2p+1 (entry e: codes e mod 8, e / 8)
+        constexpr int TPP = kThreads / PI;
+        const int p = threadIdx.x % PI, e0 = threadIdx.x / PI;
+        const float4 x = *reinterpret_cast<const float4*>(qrT + (2 * p) * kMaxHeads);
+        const float4 y = *reinterpret_cast<const float4*>(qrT + (2 * p + 1) * kMaxHeads);
+        for (int e = e0; e < Lo::EI; e += TPP) {
+          const float ca = cen[e & 7] * cI, cb = cen[e >> 3] * cI;
+          *reinterpret_cast<float4*>(lutI + (e * PI + p) * 16) =
+              make_float4(fmaf(x.x, ca, y.x * cb), fmaf(x.y, ca, y.y * cb),
+                          fmaf(x.z, ca, y.z * cb), fmaf(x.w, ca, y.w * cb));
+        }
+      } else {
+        for (int i = threadIdx.x; i < Lo::EI * PI; i += kThreads) {
+          const int pp = i % PI, e = i / PI;
+          const float4 u = NI[(e & 15) * PN + pp], v = NI[(16 + (e >> 4)) * PN + pp];
+          *reinterpret_cast<float4*>(lutI + (e * PI + pp) * 16) =
+              make_float4(u.x + v.x, u.y + v.y, u.z + v.z, u.w + v.w);
+        }
+      }
+      for (int i = threadIdx.x; i < Lo::ES * Lo::PS; i += kThreads) {
+        const int pp = i % Lo::PS, e = i / Lo::PS;
+        const float4 u = NS[(e & 15) * Lo::PS + pp], v = NS[(16 + (e >> 4)) * Lo::PS + pp];
+        *reinterpret_cast<float4*>(lutS + (e * Lo::PS + pp) * 16) =
+            make_float4(u.x + v.x, u.y + v.y, u.z + v.z, u.w + v.w);
       }
     }
     __syncthreads();
 
-    // ---------------- main loop over tiles (b2-b4)
-    uint64_t* sPP = reinterpret_cast<uint64_t*>(smem + Lo::ppair) + warp * 32 * kMaxHeads;
-    float4* sVP = reinterpret_cast<float4*>(smem + Lo::vpair) + warp * 32 * 4;
-    int it = 0;
-    for (int ts = t0; ts < t1; ts += kTile, ++it) {
-      uint8_t* cur = tiles + (Lo::STAGES == 2 ? (it & 1) * Lo::stage : 0);
-      if constexpr (Lo::STAGES == 2) {
-        if (ts + kTile < t1)
-          load_tile<MB, VB, NH4>(tiles + ((it + 1) & 1) * Lo::stage, a, kvrow + ts + kTile,
-                                 tile_count(ts + kTile));
-        cp_async_commit();
-        cp_async_wait<1>();
+    // ---------------- main loop: this warp's chunks
+    ulonglong2* sPP = reinterpret_cast<ulonglong2*>(smem + Lo::ppair) + warp * 2 * 32;
+    float4* sVP = reinterpret_cast<float4*>(smem + Lo::vpair) + warp * 4 * kVpStride;
+    const uint32_t r8 = static_cast<uint32_t>(lane & 7);
+    const bool swap = r8 >= 4;
+    const uint32_t sh = 8 * (r8 & 3);
+    uint32_t rot16[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) rot16[i] = ((r8 + i) & 7) * 16;
+
+    for (int ts = c0; ts < t1; ts += kChunkStride) {
+      // prefetch the next chunk's key bytes
+      uint32_t nkw[IB / 4], nsw[4], nnw;
+      const int tn = ts + kChunkStride;
+      if (tn < t1) load_keys(tn, nkw, nsw, nnw);
+      const int wcount = min(32, t1 - ts);
+      const bool valid = lane < wcount;
+
+      uint64_t accI[2] = {0ull, 0ull}, accS[2] = {0ull, 0ull};
+#pragma unroll
+      for (int blk = 0; blk < 2; ++blk) {
+        uint32_t R0, R1;
+        rot_block(sw4[2 * blk], sw4[2 * blk + 1], swap, sh, R0, R1);
+        block_lookups<Lo::PS * 16>(accS, R0, R1, lutS, blk, rot16);
+      }
+      if constexpr (MB != 3) {
+#pragma unroll
+        for (int blk = 0; blk < IB / 8; ++blk) {
+          uint32_t R0, R1;
+          rot_block(kw[2 * blk], kw[2 * blk + 1], swap, sh, R0, R1);
+          block_lookups<PI * 16>(accI, R0, R1, lutI, blk, rot16);
+        }
       } else {
-        if (it > 0) {
-          load_tile<MB, VB, NH4>(tiles, a, kvrow + ts, tile_count(ts));
-          cp_async_commit();
+        // bytes of two 3-bit codes: the mirror flips both codes (bit 6 set: high code >= 4)
+#pragma unroll
+        for (int blk = 0; blk < IB / 8; ++blk) {
+          uint32_t R0, R1;
+          rot_block(kw[2 * blk], kw[2 * blk + 1], swap, sh, R0, R1);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t v = ((i < 4 ? R0 : R1) >> (8 * (i & 3))) & 0xffu;
+            const int msk = static_cast<int>(v << 25) >> 31;
+            const uint32_t vc = v ^ (static_cast<uint32_t>(msk) & 0x77u);
+            const uint32_t en = (vc & 7u) | ((vc >> 1) & 0x18u);
+            lut_acc(accI, lutI + 128 * blk + en * (PI * 16) + rot16[i], sign_pair(msk));
+          }
+        }
+      }
+      const float n16 = half_lo(nw), r16 = half_hi(nw);
+      float sc[kMaxHeads];
+#pragma unroll
+      for (int j = 0; j < kMaxHeads / 2; ++j) {
+        const float2 xi = up2(accI[j]), xs = up2(accS[j]);
+        sc[2 * j] = fmaf(n16, xi.x, r16 * xs.x);
+        sc[2 * j + 1] = fmaf(n16, xi.y, r16 * xs.y);
+      }
+      if (a.scores != nullptr && valid) {
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          if (h < nh) {
+            const int hq = a.g_heads[grp][h];
+            a.scores[(static_cast<int64_t>(b) * a.n_q_heads + hq) * a.scores_ld + ts + lane] =
+                sc[h] * a.inv_scale_log2;
+          }
+        }
+      }
+      if constexpr (HAS_V) {
+        // online softmax: p pairs and this token's dequant pairs to the warp's slots
+        float p[NH];
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          const float s = (valid && h < nh) ? sc[h] : -INFINITY;
+          const float mx = warp_max(s);
+          const float mn = fmaxf(m[h], mx);
+          const float alpha = mn == -INFINITY ? 1.f : exp2f(m[h] - mn);
+          p[h] = mn == -INFINITY ? 0.f : exp2f(s - mn);
+          l[h] = fmaf(l[h], alpha, p[h]);
+          const uint64_t al = pk2(alpha, alpha);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) o[h][k] = mul2(o[h][k], al);
+          m[h] = mn;
+        }
+        {
+          float pp[kMaxHeads];  // p of the head slots, zero past NH
+#pragma unroll
+          for (int h = 0; h < kMaxHeads; ++h) pp[h] = h < NH ? p[h < NH ? h : 0] : 0.f;
+          sPP[lane] = make_ulonglong2(pk2(pp[0], pp[0]), pk2(pp[1], pp[1]));
+          if constexpr (NH > 2) sPP[32 + lane] = make_ulonglong2(pk2(pp[2], pp[2]), pk2(pp[3], pp[3]));
         }
         cp_async_wait<0>();
-      }
-      __syncthreads();
-
-      const int nk = min(kTile, t1 - ts);
-      const int wcount = max(0, min(32, nk - 32 * warp));
-      if (wcount > 0) {
-        const int my = 32 * warp + lane;
-        const bool valid = lane < wcount;
-        uint64_t accI[4] = {0ull, 0ull, 0ull, 0ull}, accS[4] = {0ull, 0ull, 0ull, 0ull};
-        // sign nibbles, rotated by `lane` nibbles: nibble k of RS[i] = (lane + 8i + k) mod 32
+        __syncwarp();
         {
-          const uint32_t* sr = reinterpret_cast<const uint32_t*>(cur + Lo::o_sgn + my * 16);
-          const int q = lane >> 3, sh = 4 * (lane & 7);
-          uint32_t w[4];
+          // v_hat = mn16 + code * s16 = f * (16 s16) + (mn16 - 16 s16), f = 1 + code / 16
+          const uint4 par = *reinterpret_cast<const uint4*>(wslot + Lo::o_vp + lane * 16);
+          const uint32_t pw[4] = {par.x, par.y, par.z, par.w};
 #pragma unroll
-          for (int i = 0; i < 4; ++i) w[i] = sr[(q + i) & 3];
-          const uint8_t* lb = lutS + lane * 16;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t R = __funnelshift_r(w[i], w[(i + 1) & 3], sh);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              nib_step<NH4, Lo::HALF_S, Lo::PDS * 16>(accS, R, k, lb, 8 * i + k);
+          for (int g = 0; g < 4; ++g) {
+            const float mnv = half_lo(pw[g]), scv = half_hi(pw[g]);
+            const float s16 = 16.f * scv, cc = fmaf(-16.f, scv, mnv);
+            sVP[g * kVpStride + lane] = make_float4(s16, s16, cc, cc);
           }
         }
-        if constexpr (MB == 2 || MB == 1) {
-          // index nibbles, rotated by `lane` nibbles
-          constexpr int NW = IB / 4;       // 8 words (2-bit) or 4 words (1-bit)
-          const uint32_t* kr = reinterpret_cast<const uint32_t*>(cur + Lo::o_idx + my * IB);
-          const int q = lane >> 3, sh = 4 * (lane & 7);
-          uint32_t w[NW];
+        __syncwarp();
+
+        // P.V: token 2 jj + hw of the chunk per step, 8 channels per lane (group j16 / 4)
+        const int hw = lane >> 4, j16 = lane & 15, vg = j16 >> 2;
+#pragma unroll 2
+        for (int jj = 0; 2 * jj < wcount; ++jj) {
+          const int tok = 2 * jj + hw;
+          if (tok < wcount) {
+            const float4 dq = sVP[vg * kVpStride + tok];
+            const uint64_t S16 = pk2(dq.x, dq.y), CC = pk2(dq.z, dq.w);
+            uint32_t cw[8];
+            if constexpr (VB == 2) {
+              const uint32_t c16 = reinterpret_cast<const uint16_t*>(wslot + Lo::o_vq + tok * 32)[j16];
 #pragma unroll
-          for (int i = 0; i < NW; ++i) w[i] = kr[(q + i) % NW];
-          const uint8_t* lb = lutI + lane * 16;
+              for (int k = 0; k < 8; ++k) cw[k] = (c16 << (19 - 2 * k)) & 0x00180000u;
+            } else {
+              const uint32_t c32 = reinterpret_cast<const uint32_t*>(wslot + Lo::o_vq + tok * 64)[j16];
 #pragma unroll
-          for (int i = 0; i < NW; ++i) {
-            const uint32_t R = __funnelshift_r(w[i], w[(i + 1) % NW], sh);
+              for (int k = 0; k < 8; ++k)
+                cw[k] = (k < 5 ? (c32 << (19 - 4 * k)) : (c32 >> (4 * k - 19))) & 0x00780000u;
+            }
+            uint64_t v[4];
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              nib_step<NH4, Lo::HALF_I, PDI * 16>(accI, R, k, lb, 8 * i + k);
-          }
-        } else {
-          // 64 index bytes (two 3-bit codes in nibbles), rotated by `lane` bytes
-          const uint32_t* kr = reinterpret_cast<const uint32_t*>(cur + Lo::o_idx + my * IB);
-          const int q = lane >> 2, sh = 8 * (lane & 3);
-          uint32_t w[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) w[i] = kr[(q + i) & 15];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const uint32_t R = __funnelshift_r(w[i], w[(i + 1) & 15], sh);
+            for (int k = 0; k < 4; ++k)
+              v[k] = fma2(pk2(__uint_as_float(0x3f800000u | cw[2 * k]), __uint_as_float(0x3f800000u | cw[2 * k + 1])), S16, CC);
+            const ulonglong2 p01 = sPP[tok];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const int s = 4 * i + k;
-              const uint32_t v = (R >> (8 * k)) & 0xffu;
-              const int msk = static_cast<int>(v << 25) >> 31;          // bit 6: high code >= 4
-              const uint32_t vc = v ^ (static_cast<uint32_t>(msk) & 0x77u);
-              const uint32_t en = (vc & 7u) | ((vc >> 1) & 0x18u);
-              const uint32_t p6 = static_cast<uint32_t>((lane + s) & 63);
-              lut_acc<NH4, Lo::HALF_I>(accI, lutI + (en * PDI + p6) * 16, sign_pair(msk));
+              o[0][k] = fma2(p01.x, v[k], o[0][k]);
+              if constexpr (NH > 1) o[1][k] = fma2(p01.y, v[k], o[1][k]);
+            }
+            if constexpr (NH > 2) {
+              const ulonglong2 p23 = sPP[32 + tok];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                o[2][k] = fma2(p23.x, v[k], o[2][k]);
+                if constexpr (NH > 3) o[3][k] = fma2(p23.y, v[k], o[3][k]);
+              }
             }
           }
         }
-        const uint32_t nn = reinterpret_cast<const uint32_t*>(cur + Lo::o_nrm)[my];
-        const float n16 = half_lo(nn), r16 = half_hi(nn);
-        float sc[NH];
-#pragma unroll
-        for (int j = 0; j < NH / 2; ++j) {
-          const float2 xi = up2(accI[j]), xs = up2(accS[j]);
-          sc[2 * j] = fmaf(n16, xi.x, r16 * xs.x);
-          sc[2 * j + 1] = fmaf(n16, xi.y, r16 * xs.y);
-        }
-        if (a.scores != nullptr && valid) {
-#pragma unroll
-          for (int h = 0; h < NH; ++h) {
-            if (h < nh) {
-              const int hq = a.g_heads[grp][h];
-              a.scores[(static_cast<int64_t>(b) * a.n_q_heads + hq) * a.scores_ld + ts + my] =
-                  sc[h] * a.inv_scale_log2;
-            }
-          }
-        }
-        if constexpr (HAS_V) {
-          // online softmax (b3): p pairs and this token's dequant pairs to shared
-          float p[NH];
-#pragma unroll
-          for (int h = 0; h < NH; ++h) {
-            const float s = (valid && h < nh) ? sc[h] : -INFINITY;
-            const float mx = warp_max(s);
-            const float mn = fmaxf(m[h], mx);
-            const float alpha = mn == -INFINITY ? 1.f : exp2f(m[h] - mn);
-            p[h] = mn == -INFINITY ? 0.f : exp2f(s - mn);
-            l[h] = fmaf(l[h], alpha, p[h]);
-            const uint64_t al = pk2(alpha, alpha);
-            o[h][0] = mul2(o[h][0], al);
-            o[h][1] = mul2(o[h][1], al);
-            m[h] = mn;
-          }
-          uint64_t* myp = sPP + lane * kMaxHeads;
-#pragma unroll
-          for (int h = 0; h < NH; h += 2)
-            *reinterpret_cast<ulonglong2*>(myp + h) = make_ulonglong2(pk2(p[h], p[h]), pk2(p[h + 1], p[h + 1]));
-          {
-            // v_hat = mn16 + code * s16 = f * (16 s16) + (mn16 - 16 s16), f = 1 + code / 16
-            const uint4 par = *reinterpret_cast<const uint4*>(cur + Lo::o_vp + my * 16);
-            const uint32_t pw[4] = {par.x, par.y, par.z, par.w};
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              const float mnv = half_lo(pw[g]), scv = half_hi(pw[g]);
-              const float s16 = 16.f * scv, cc = fmaf(-16.f, scv, mnv);
-              sVP[lane * 4 + g] = make_float4(s16, s16, cc, cc);
-            }
-          }
-          __syncwarp();
-
-          // P.V (b4): lane owns channels 4 lane .. 4 lane + 3 (group lane / 8), one token a step
-          const int vg = lane >> 3;
-#pragma unroll 2
-          for (int i = 0; i < wcount; ++i) {
-            const int tok = 32 * warp + i;
-            const float4 dq = sVP[i * 4 + vg];
-            const uint64_t S16 = pk2(dq.x, dq.y), CC = pk2(dq.z, dq.w);
-            uint32_t c0, c1, c2, c3;
-            if constexpr (VB == 2) {
-              const uint32_t by = cur[Lo::o_vq + tok * 32 + lane];
-              c0 = by << 19; c1 = by << 17; c2 = by << 15; c3 = by << 13;
-              c0 &= 0x00180000u; c1 &= 0x00180000u; c2 &= 0x00180000u; c3 &= 0x00180000u;
-            } else {
-              const uint32_t hw = reinterpret_cast<const uint16_t*>(cur + Lo::o_vq + tok * 64)[lane];
-              c0 = (hw << 19) & 0x00780000u; c1 = (hw << 15) & 0x00780000u;
-              c2 = (hw << 11) & 0x00780000u; c3 = (hw << 7) & 0x00780000u;
-            }
-            const uint64_t f01 = pk2(__uint_as_float(0x3f800000u | c0), __uint_as_float(0x3f800000u | c1));
-            const uint64_t f23 = pk2(__uint_as_float(0x3f800000u | c2), __uint_as_float(0x3f800000u | c3));
-            const uint64_t v01 = fma2(f01, S16, CC), v23 = fma2(f23, S16, CC);
-            const uint64_t* pp = sPP + i * kMaxHeads;
-#pragma unroll
-            for (int h = 0; h < NH; h += 2) {
-              const ulonglong2 ph = *reinterpret_cast<const ulonglong2*>(pp + h);
-              o[h][0] = fma2(ph.x, v01, o[h][0]);
-              o[h][1] = fma2(ph.x, v23, o[h][1]);
-              o[h + 1][0] = fma2(ph.y, v01, o[h + 1][0]);
-              o[h + 1][1] = fma2(ph.y, v23, o[h + 1][1]);
-            }
-          }
-          __syncwarp();
-        }
+        __syncwarp();
+        if (tn < t1) load_values(tn);
       }
-      __syncthreads();
+#pragma unroll
+      for (int i = 0; i < IB / 4; ++i) kw[i] = nkw[i];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sw4[i] = nsw[i];
+      nw = nnw;
     }
     cp_async_wait<0>();
   }
+  grid_dependency_wait();  // (CTAs past the longest sequence skipped the wait above)
 
   if constexpr (!HAS_V) return;
 
-  // ---------------- merge the 8 warps of this CTA (b5)
+  // ---------------- merge the warps of this CTA
   __syncthreads();
-  float* sM = reinterpret_cast<float*>(tiles);  // [warp][head][kPartStride]
+  float* sM = reinterpret_cast<float*>(smem + Lo::wv);  // [warp][head][kPartStride]
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
+    // the two half-warps hold disjoint tokens of the same channels
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 v = up2(o[h][k]);
+      o[h][k] = add2(o[h][k], pk2(__shfl_xor_sync(kFull, v.x, 16), __shfl_xor_sync(kFull, v.y, 16)));
+    }
     if (h < nh) {
       const float lt = warp_sum(l[h]);
       float* dst = sM + (warp * kMaxHeads + h) * kPartStride;
       if (lane == 0) { dst[0] = m[h]; dst[1] = lt; }
-      const float2 v0 = up2(o[h][0]), v1 = up2(o[h][1]);
-      *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = make_float4(v0.x, v0.y, v1.x, v1.y);
+      if (lane < 16) {
+        const float2 v0 = up2(o[h][0]), v1 = up2(o[h][1]), v2 = up2(o[h][2]), v3 = up2(o[h][3]);
+        *reinterpret_cast<float4*>(dst + 4 + 8 * lane) = make_float4(v0.x, v0.y, v1.x, v1.y);
+        *reinterpret_cast<float4*>(dst + 8 + 8 * lane) = make_float4(v2.x, v2.y, v3.x, v3.y);
+      }
     }
   }
   __syncthreads();
@@ -553,11 +600,11 @@ k_decode(const __grid_constant__ DecodeArgs a) {
     const int h = warp, hq = a.g_heads[grp][h];
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) M = fmaxf(M, sM[(w * kMaxHeads + h) * kPartStride]);
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sM[(w * kMaxHeads + h) * kPartStride]);
     float Lsum = 0.f, O[4] = {0.f, 0.f, 0.f, 0.f};
     if (M != -INFINITY) {
 #pragma unroll
-      for (int w = 0; w < 8; ++w) {
+      for (int w = 0; w < kWarps; ++w) {
         const float* src = sM + (w * kMaxHeads + h) * kPartStride;
         if (src[0] == -INFINITY) continue;
         const float f = exp2f(src[0] - M);
@@ -601,76 +648,97 @@ k_decode(const __grid_constant__ DecodeArgs a) {
   __syncthreads();
   if (!sLast) return;
   __threadfence();
-  // one warp per head, heads in parallel: lanes read the split maxima and sums (lane = split),
-  // then the weighted partial outputs are loaded 16 splits at a time (independent loads)
-  if (warp < nh) {
-    const int h = warp, hq = a.g_heads[grp][h];
-    const float* base = a.part + (static_cast<int64_t>(b) * a.n_q_heads + hq) * a.n_splits * kPartStride;
-    float mloc = -INFINITY;
-    for (int s = lane; s < a.n_splits; s += 32) mloc = fmaxf(mloc, __ldcg(base + s * kPartStride));
-    const float M = warp_max(mloc);
-    float Lsum = 0.f, O[4] = {0.f, 0.f, 0.f, 0.f};
-    if (M != -INFINITY) {
-      for (int s0 = 0; s0 < a.n_splits; s0 += 32) {
-        const int s = s0 + lane;
-        float f = 0.f;
-        if (s < a.n_splits) {
-          const float ms = __ldcg(base + s * kPartStride);
-          const float lsv = __ldcg(base + s * kPartStride + 1);
-          if (ms != -INFINITY) {
-            f = exp2f(ms - M);
-            Lsum = fmaf(f, lsv, Lsum);
-          }
-        }
-        const int cnt = min(32, a.n_splits - s0);
-        const float* blk = base + s0 * kPartStride + 4 + 4 * lane;
-        int j = 0;
-        for (; j + 16 <= cnt; j += 16) {
-          float4 ov[16];
+  // Every (head, split) pair's maximum and sum, then every (head, channel quad, split slice)
+  // item's weighted partial outputs, are loaded by all threads at once (one round trip each);
+  // the slices are summed in shared memory.
+  {
+    const int S = a.n_splits;
+    float* sMx = reinterpret_cast<float*>(smem + Lo::wv);   // [head][S] split maxima
+    float* sLs = sMx + kMaxHeads * 256;                      // [head][S] split sums
+    float* sF = sLs + kMaxHeads * 256;                       // [head][S] weights
+    float* sHd = sF + kMaxHeads * 256;                       // [head]: 1 / total sum
+    float4* sAcc = reinterpret_cast<float4*>(sHd + 16);      // [slice][head][32]
+    const float* base = a.part + static_cast<int64_t>(b) * a.n_q_heads * S * kPartStride;
+    for (int i = threadIdx.x; i < nh * S; i += kThreads) {
+      const int h = i / S, sp = i - h * S;
+      const float* src = base + (static_cast<int64_t>(a.g_heads[grp][h]) * S + sp) * kPartStride;
+      sMx[h * 256 + sp] = __ldcg(src);
+      sLs[h * 256 + sp] = __ldcg(src + 1);
+    }
+    __syncthreads();
+    if (warp < nh) {
+      const int h = warp;
+      float mloc = -INFINITY;
+      for (int sp = lane; sp < S; sp += 32) mloc = fmaxf(mloc, sMx[h * 256 + sp]);
+      const float M = warp_max(mloc);
+      float lsum = 0.f;
+      for (int sp = lane; sp < S; sp += 32) {
+        const float ms = sMx[h * 256 + sp];
+        const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : exp2f(ms - M);
+        sF[h * 256 + sp] = f;
+        lsum = fmaf(f, sLs[h * 256 + sp], lsum);
+      }
+      lsum = warp_sum(lsum);
+      if (lane == 0) sHd[h] = lsum > 0.f ? 1.f / lsum : 0.f;
+    }
+    __syncthreads();
+    const int G = kThreads / (32 * nh);  // split slices
+    if (threadIdx.x < G * 32 * nh) {
+      const int h = threadIdx.x / (32 * G), r = threadIdx.x - h * 32 * G;
+      const int qd = r & 31, g = r >> 5;
+      const float* src = base + static_cast<int64_t>(a.g_heads[grp][h]) * S * kPartStride + 4 + 4 * qd;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      int sp = g;
+      for (; sp + 3 * G < S; sp += 4 * G) {
+        float4 v[4];
 #pragma unroll
-          for (int u = 0; u < 16; ++u) ov[u] = __ldcg(reinterpret_cast<const float4*>(blk + (j + u) * kPartStride));
+        for (int u = 0; u < 4; ++u) v[u] = __ldcg(reinterpret_cast<const float4*>(src + static_cast<int64_t>(sp + u * G) * kPartStride));
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const float fj = __shfl_sync(kFull, f, j + u);
-            O[0] = fmaf(fj, ov[u].x, O[0]);
-            O[1] = fmaf(fj, ov[u].y, O[1]);
-            O[2] = fmaf(fj, ov[u].z, O[2]);
-            O[3] = fmaf(fj, ov[u].w, O[3]);
-          }
-        }
-        for (; j < cnt; ++j) {
-          const float fj = __shfl_sync(kFull, f, j);
-          const float4 ov = __ldcg(reinterpret_cast<const float4*>(blk + j * kPartStride));
-          O[0] = fmaf(fj, ov.x, O[0]);
-          O[1] = fmaf(fj, ov.y, O[1]);
-          O[2] = fmaf(fj, ov.z, O[2]);
-          O[3] = fmaf(fj, ov.w, O[3]);
+        for (int u = 0; u < 4; ++u) {
+          const float f = sF[h * 256 + sp + u * G];
+          acc.x = fmaf(f, v[u].x, acc.x); acc.y = fmaf(f, v[u].y, acc.y);
+          acc.z = fmaf(f, v[u].z, acc.z); acc.w = fmaf(f, v[u].w, acc.w);
         }
       }
-      Lsum = warp_sum(Lsum);
+      for (; sp < S; sp += G) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(src + static_cast<int64_t>(sp) * kPartStride));
+        const float f = sF[h * 256 + sp];
+        acc.x = fmaf(f, v.x, acc.x); acc.y = fmaf(f, v.y, acc.y);
+        acc.z = fmaf(f, v.z, acc.z); acc.w = fmaf(f, v.w, acc.w);
+      }
+      sAcc[(g * kMaxHeads + h) * 32 + qd] = acc;
     }
-    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-    const int64_t orow = (static_cast<int64_t>(b) * a.n_q_heads + hq) * kD + 4 * lane;
-    if (a.out_f32) {
-      *reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow) =
-          make_float4(O[0] * inv, O[1] * inv, O[2] * inv, O[3] * inv);
-    } else {
-      __nv_bfloat162 lo = __floats2bfloat162_rn(O[0] * inv, O[1] * inv);
-      __nv_bfloat162 hi = __floats2bfloat162_rn(O[2] * inv, O[3] * inv);
-      uint2 pk;
-      pk.x = *reinterpret_cast<uint32_t*>(&lo);
-      pk.y = *reinterpret_cast<uint32_t*>(&hi);
-      *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + orow) = pk;
+    __syncthreads();
+    if (threadIdx.x < 32 * nh) {
+      const int h = threadIdx.x >> 5, qd = threadIdx.x & 31, hq = a.g_heads[grp][h];
+      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int g = 0; g < G; ++g) {
+        const float4 v = sAcc[(g * kMaxHeads + h) * 32 + qd];
+        O.x += v.x; O.y += v.y; O.z += v.z; O.w += v.w;
+      }
+      const float inv = sHd[h];
+      const int64_t orow = (static_cast<int64_t>(b) * a.n_q_heads + hq) * kD + 4 * qd;
+      if (a.out_f32) {
+        *reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow) =
+            make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
+      } else {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(O.x * inv, O.y * inv);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(O.z * inv, O.w * inv);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + orow) = pk;
+      }
     }
   }
   if (threadIdx.x == 0) a.counters[static_cast<int64_t>(b) * a.n_q_heads + a.g_heads[grp][0]] = 0;
 }
 
-template <int MB, int VB, int NH4>
+template <int MB, int VB, int NH>
 tq_status run_decode(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
-  constexpr int smem = Lay<MB, VB, NH4>::total;
+  constexpr int smem = Lay<MB, VB>::total;
   static_assert(smem <= 227 * 1024, "decode shared memory budget");
-  auto kern = k_decode<MB, VB, NH4>;
+  auto kern = k_decode<MB, VB, NH>;
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
@@ -678,17 +746,29 @@ tq_status run_decode(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
       return TQ_ECUDA;
     configured = true;
   }
-  kern<<<grid, kThreads, smem, st>>>(a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return TQ_ECUDA;
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ECUDA;
 }
 
 template <int MB, int VB>
 tq_status run_decode_nh(const DecodeArgs& a, dim3 grid, int max_heads, cudaStream_t st) {
-  return max_heads <= 4 ? run_decode<MB, VB, 1>(a, grid, st) : run_decode<MB, VB, 2>(a, grid, st);
+  if (max_heads <= 2) return run_decode<MB, VB, 2>(a, grid, st);
+  if (max_heads == 3) return run_decode<MB, VB, 3>(a, grid, st);
+  return run_decode<MB, VB, 4>(a, grid, st);
 }
 
 int max_splits_for(int capacity) {
-  const int s = (capacity + kTile - 1) / kTile;
+  const int s = (capacity + 255) / 256;
   return s < 1 ? 1 : (s > 256 ? 256 : s);
 }
 
@@ -726,7 +806,7 @@ tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* c, const void*
   a.scale_log2 = scale * 1.4426950408889634074f;
   a.inv_scale_log2 = 1.f / a.scale_log2;
 
-  // head groups: the query heads of each KV head, in balanced groups of at most 8
+  // head groups: the query heads of each KV head, in balanced groups of at most 4
   int n_groups = 0, max_heads = 0;
   for (int kv = 0; kv < c->n_kv_heads; ++kv) {
     int heads[1024];
@@ -753,25 +833,28 @@ tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* c, const void*
   for (int b = 0; b < c->batch; ++b) max_len = c->len_host[b] > max_len ? c->len_host[b] : max_len;
   if (max_len == 0 && out == nullptr) return TQ_OK;
 
-  // split count: minimise (CTAs per SM) x (tokens per split + per-CTA set-up) + the final
-  // combine; CTAs sharing an SM share its issue slots, so they count as serial work
+  // split count: one CTA per SM; minimise waves x (tokens per split + per-CTA set-up) + the
+  // final combine (its loads grow with the number of splits). A few SMs are left out of the
+  // first wave so that an append kernel still resident on them does not hold back a CTA of
+  // this grid when it starts early (programmatic dependent launch).
   int dev = 0;
   cudaGetDevice(&dev);
-  const int sms = sm_count(dev);
+  const int sms = std::max(1, sm_count(dev) - 4);
   const int pairs = c->batch * n_groups;
   const int cap_splits = max_splits_for(c->capacity);
   int best = 1;
   double best_cost = 1e300;
-  const int max_try = std::max(1, std::min(cap_splits, (max_len + 127) / 128));
+  const int max_try = std::max(1, std::min(cap_splits, (max_len + 255) / 256));
   for (int s = 1; s <= max_try; ++s) {
     const int tps = ((max_len + s - 1) / s + 31) & ~31;
     const int used = (max_len + tps - 1) / tps;
     if (used != s) continue;
     const double waves = std::ceil(static_cast<double>(pairs) * s / sms);
-    const double cost = waves * (tps + 256.0) + (s > 1 ? 4.0 * s : 0.0);
+    const double cost = waves * (tps + 512.0) + (s > 1 ? 8.0 * s : 0.0);
     if (cost < best_cost - 1e-9) { best_cost = cost; best = s; }
   }
   a.n_splits = best;
+  a.max_len = max_len;
   a.tokens_per_split = std::max(32, ((max_len + best - 1) / best + 31) & ~31);
   if (decode_workspace_bytes(c->batch, n_q_heads, c->capacity) > workspace_bytes) return TQ_EINVAL;
   const size_t parts = static_cast<size_t>(c->batch) * n_q_heads * cap_splits * kPartStride * sizeof(float);
