@@ -128,7 +128,8 @@ class ClockSampler:
         return {"sm_mhz": med, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sms)}
 
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend=None):
+    """One process per GPU (torchrun env). NCCL on GPUs; gloo when asked (CPU tests)."""
     import torch
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -136,40 +137,55 @@ def dist_setup(n_gpus):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        backend = backend or "nccl"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
+    elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return rank, world, local
 
 
-def barrier(world):
+def _sync_device():
     import torch
+    if torch.cuda.is_available() and torch.cuda.is_initialized():
+        torch.cuda.synchronize()
+
+
+def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    _sync_device()
+
+
+def _all_reduce(x: float, world: int, op: str) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], device=dev, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
 
 
 def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return _all_reduce(x, world, "max")
 
 
 def sum_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return _all_reduce(x, world, "sum")
+
+
+def replica_throughput(units: float, ms: float, world: int):
+    """Whole-job throughput of independent replicas: the units all ranks processed over the
+    slowest rank's time. Returns (units per second, max ms over ranks)."""
+    ms_max = max_over_ranks(ms, world)
+    return sum_over_ranks(units, world) / (ms_max / 1e3), ms_max
 
 
 # ------------------------------------------------------------------------------ tq arm
@@ -253,9 +269,7 @@ def run_tq(args):
     dec_ms = [b_.elapsed_time(c) for _, b_, c in ev]
     tot_ms = sum(step_ms)
     keys_scored = float(sum(Hq * L for L in lens) * B)
-    tot_ms_max = max_over_ranks(tot_ms, world)
-    keys_all = sum_over_ranks(keys_scored, world)
-    value = keys_all / (tot_ms_max / 1e3)
+    value, tot_ms_max = replica_throughput(keys_scored, tot_ms, world)
     dec_avg_ms = sum(dec_ms) / len(dec_ms)
     mean_len = sum(lens) / len(lens)
     dec_bytes = (B * Hkv * mean_len * (key_bytes(WL["key_bits"]) + value_bytes(WL["value_bits"]))
@@ -366,7 +380,7 @@ def bench_quantize(tq, torch, dev, world, peak, peak_kind, rows=1 << 22, reps=5,
     lay = qs[0].layout
     out_bytes = lay["idx_bytes"] + lay["sign_bytes"] + 2 * lay["n_norms"]
     gbs = n * (256 + out_bytes) / (ms / 1e3) / 1e9
-    kernel = {"prod": f"k_keys_prod_tc<{bits - 1}>", "mse": f"k_keys_full<mse,{bits}>",
+    kernel = {"prod": f"k_keys_tc<prod,{bits - 1}>", "mse": f"k_keys_tc<mse,{bits}>",
               "grouped": f"k_keys_grouped<{bits}>"}[mode]
     del xs, planes
     torch.cuda.empty_cache()

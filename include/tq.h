@@ -222,6 +222,12 @@ tq_status tq_decode_attention_noalloc(const tq_quantizer* q, const tq_kv_cache* 
  * all streams. */
 tq_status tq_sync_status(void* stream);
 
+/* Diagnostic of the error path above: launches on `stream` a one-thread kernel that waits on
+ * an mbarrier phase nothing completes and gives up after `limit_us` microseconds
+ * (1 .. 2000000; else TQ_EINVAL, nothing launched), recording the timeout in the device flag
+ * so that the next tq_sync_status returns TQ_ETIMEOUT. No device fault is involved. */
+tq_status tq_selftest_bounded_wait(uint32_t limit_us, void* stream);
+
 const char* tq_status_string(tq_status s);
 int tq_abi_version(void);
 

@@ -30,7 +30,7 @@ D = 128
 EXPORTED = ["tq_build_codebook", "tq_free", "tq_key_layout", "tq_host_tables",
             "tq_quantize_keys", "tq_quantize_values", "tq_append", "tq_decode_workspace_bytes",
             "tq_decode_attention", "tq_decode_attention_noalloc", "tq_sync_status",
-            "tq_status_string", "tq_abi_version"]
+            "tq_selftest_bounded_wait", "tq_status_string", "tq_abi_version"]
 
 
 class KeyLayout(ctypes.Structure):
@@ -89,6 +89,8 @@ _lib.tq_abi_version.argtypes = []
 _lib.tq_abi_version.restype = c_int
 _lib.tq_sync_status.argtypes = [c_void_p]
 _lib.tq_sync_status.restype = c_int
+_lib.tq_selftest_bounded_wait.argtypes = [ctypes.c_uint32, c_void_p]
+_lib.tq_selftest_bounded_wait.restype = c_int
 
 
 class TQError(RuntimeError):
@@ -108,6 +110,14 @@ def tq_status_string(status: int) -> str:
 
 def tq_abi_version() -> int:
     return _lib.tq_abi_version()
+
+
+def tq_selftest_bounded_wait(limit_us: int, stream=None) -> None:
+    """Launch the diagnostic kernel whose bounded wait runs out after limit_us microseconds;
+    the next tq_sync_status raises TQError(TQ_ETIMEOUT)."""
+    in_range = 0 < limit_us <= 2_000_000   # out-of-range limits are rejected on the host
+    _check(_lib.tq_selftest_bounded_wait(limit_us, _stream(stream) if in_range else None),
+           "tq_selftest_bounded_wait")
 
 
 def tq_sync_status(stream=None) -> None:

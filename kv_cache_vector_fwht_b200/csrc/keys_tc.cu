@@ -114,10 +114,13 @@ __device__ __forceinline__ void store_signs(const TcKeyArgs& a, uint32_t tlane, 
         make_uint4(sg[0], sg[1], sg[2], sg[3]);
 }
 
-template <int MB>
+// PROD: prod keys (MB = bits - 1, residual + QJL on tcgen05); else mse keys (MB = bits,
+// indices and the norm only; the accumulator columns only park the rotated row).
+template <bool PROD, int MB>
 __global__ void __launch_bounds__(128, 2)
-    k_keys_prod_tc(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ TcKeyArgs a) {
+    k_keys_tc(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ TcKeyArgs a) {
   constexpr int NL = 1 << MB;
+  constexpr uint32_t TCOLS = PROD ? kTmemCols : 128u;
   constexpr int W = storage_width_c(MB);
   constexpr int NW = 4 * W;       // index words per row
   constexpr int GP = 32 / W;      // pairs per decision group: one index word per half
@@ -140,7 +143,7 @@ __global__ void __launch_bounds__(128, 2)
   const int64_t n_local = (a.n_tiles - blockIdx.x + grid - 1) / grid;  // grid <= n_tiles
 
   if (warp == 0) {
-    tmem_alloc(&tslot, kTmemCols);
+    tmem_alloc(&tslot, TCOLS);
     tmem_relinquish();
   }
   if (tid == 0) {
@@ -158,8 +161,8 @@ __global__ void __launch_bounds__(128, 2)
   const uint32_t tlane = tbase + (static_cast<uint32_t>(warp * 32) << 16);
 
   if (tid == 0) {
-    mbar_expect_tx(&bar_b, kBBytes + 256);
-    bulk_g2s(sB, tab->s_umma, kBBytes, &bar_b);
+    mbar_expect_tx(&bar_b, (PROD ? kBBytes : 0) + 256);
+    if constexpr (PROD) bulk_g2s(sB, tab->s_umma, kBBytes, &bar_b);
     bulk_g2s(smem + kMaskOff, tab->pair_mask, 256, &bar_b);
     for (int k = 0; k < 2 && k < n_local; ++k) {
       const int row0 = static_cast<int>((blockIdx.x + k * grid) * kTile);
@@ -240,7 +243,7 @@ __global__ void __launch_bounds__(128, 2)
     const float n16f = __half2float(n16);
 
     // ---- previous tile: sign bits of its QJL product
-    if (k > 0) {
+    if (PROD && k > 0) {
       if (ok) ok = mbar_wait_ns(&bar_mma, static_cast<uint32_t>((k - 1) & 1), kWaitNs);
       tc_fence_after();
       store_signs(a, tlane, prev_valid, prev_zero, a.row_base + prev_row);
@@ -266,7 +269,7 @@ __global__ void __launch_bounds__(128, 2)
 #pragma unroll
     for (int t = 0; t < NL - 1; ++t) T[t] = n > 0.f ? thr[t] * n : thr[t];
     const uint32_t ex = (__float_as_uint(n) >> 23) & 0xffu;
-    const float scl = __uint_as_float((ex >= 10u ? 264u - ex : 254u) << 23);
+    const float scl = PROD ? __uint_as_float((ex >= 10u ? 264u - ex : 254u) << 23) : 1.f;
     // The centroid term of code c is ncs[0] + sum_{t < c} dcs[t]: a multiply-add per exact
     // 0/1 compare (its rounding moves rho by about an ulp, far inside the parity margins).
     float ncs[NL];
@@ -309,10 +312,11 @@ __global__ void __launch_bounds__(128, 2)
             const float2 th = up2(T2[t]);
             const uint64_t ind = pk2(gt_one(__uint_as_float(yv[2 * i]), th.x),
                                      gt_one(__uint_as_float(yv[2 * i + 1]), th.y));
-            c2 = fma2(ind, dcs2[t], c2);
+            if constexpr (PROD) c2 = fma2(ind, dcs2[t], c2);
             if (pi < GP / 2) wa = fma2(ind, kw2, wa);
             else wb = fma2(ind, kw2, wb);
           }
+          if constexpr (!PROD) continue;
           const uint64_t r = fma2(y2, scl2, c2);
           racc[pi & 3] = fma2(r, r, racc[pi & 3]);
           // Veltkamp split: hi keeps the top 11 significant bits (exact in fp16 for |r| < 2^15),
@@ -325,7 +329,8 @@ __global__ void __launch_bounds__(128, 2)
           lw[pi] = h2_bits(lv.x, lv.y);
         }
       }
-      if constexpr (GP == 8) {
+      if constexpr (!PROD) {
+      } else if constexpr (GP == 8) {
         tmem_st8(tlane + 128 + GP * g, *reinterpret_cast<uint32_t(*)[8]>(hw));
         tmem_st8(tlane + 192 + GP * g, *reinterpret_cast<uint32_t(*)[8]>(lw));
       } else {
@@ -356,8 +361,11 @@ __global__ void __launch_bounds__(128, 2)
       for (int w = 0; w < NW; w += 4)
         dst[w / 4] = make_uint4(sCode[w * kTile + tid], sCode[(w + 1) * kTile + tid],
                                 sCode[(w + 2) * kTile + tid], sCode[(w + 3) * kTile + tid]);
-      *reinterpret_cast<uint32_t*>(a.nrm + orow * 2) =
-          static_cast<uint32_t>(half_bits(n16)) | (static_cast<uint32_t>(half_bits(r16)) << 16);
+      if constexpr (PROD)
+        *reinterpret_cast<uint32_t*>(a.nrm + orow * 2) =
+            static_cast<uint32_t>(half_bits(n16)) | (static_cast<uint32_t>(half_bits(r16)) << 16);
+      else
+        a.nrm[orow] = half_bits(n16);
     }
     prev_row = row;
     prev_valid = valid;
@@ -371,12 +379,14 @@ __global__ void __launch_bounds__(128, 2)
       if (ok) ok = mbar_wait_ns(&bar_a, static_cast<uint32_t>(k & 1), kWaitNs);
       tc_fence_after();
       if (ok) {
+        if constexpr (PROD) {
 #pragma unroll
-        for (int s = 0; s < 16; ++s) {
-          const uint64_t bdesc = umma_desc(smem_u32(sB) + (s & 7) * 256, 128, 2048);
-          umma_f16_ts(tbase, tbase + 128 + 8 * s, bdesc, idesc, s > 0 ? 1u : 0u);
+          for (int s = 0; s < 16; ++s) {
+            const uint64_t bdesc = umma_desc(smem_u32(sB) + (s & 7) * 256, 128, 2048);
+            umma_f16_ts(tbase, tbase + 128 + 8 * s, bdesc, idesc, s > 0 ? 1u : 0u);
+          }
+          umma_commit(&bar_mma);
         }
-        umma_commit(&bar_mma);
         if (k + 2 < n_local) {
           const int row0 = static_cast<int>((tile + 2 * grid) * kTile);
           mbar_expect_tx(&bar_x[b], kXBuf);
@@ -387,7 +397,7 @@ __global__ void __launch_bounds__(128, 2)
     }
   }
 
-  if (n_local > 0) {
+  if (PROD && n_local > 0) {
     if (ok) ok = mbar_wait_ns(&bar_mma, static_cast<uint32_t>((n_local - 1) & 1), kWaitNs);
     tc_fence_after();
     if (ok) store_signs(a, tlane, prev_valid, prev_zero, a.row_base + prev_row);
@@ -397,7 +407,7 @@ __global__ void __launch_bounds__(128, 2)
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tbase, kTmemCols);
+    tmem_dealloc(tbase, TCOLS);
   }
 }
 
@@ -414,9 +424,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int MB>
+template <bool PROD, int MB>
 tq_status run_tc(const CUtensorMap& tmap, const TcKeyArgs& a, cudaStream_t st) {
-  auto kern = k_keys_prod_tc<MB>;
+  auto kern = k_keys_tc<PROD, MB>;
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
@@ -437,7 +447,7 @@ tq_status run_tc(const CUtensorMap& tmap, const TcKeyArgs& a, cudaStream_t st) {
 __device__ int g_tq_device_error = 0;
 
 bool keys_tc_ok(const tq_quantizer* q, int dtype) {
-  return q->mode == TQ_MODE_PROD && dtype == TQ_BF16 && q->bits >= 2 && q->bits <= 4 &&
+  return (q->mode == TQ_MODE_PROD || q->mode == TQ_MODE_MSE) && dtype == TQ_BF16 &&
          encode_fn() != nullptr;
 }
 
@@ -464,15 +474,40 @@ tq_status launch_keys_tc(const tq_quantizer* q, const void* x, int64_t n_rows, i
       return TQ_ECUDA;
     TcKeyArgs a{nr, r0, (nr + kTile - 1) / kTile, q->dev, out.idx, out.signs, out.norms, map, err};
     tq_status s;
-    switch (q->bits) {
-      case 2: s = run_tc<1>(tmap, a, st); break;
-      case 3: s = run_tc<2>(tmap, a, st); break;
-      case 4: s = run_tc<3>(tmap, a, st); break;
+    switch ((q->mode == TQ_MODE_PROD ? 8 : 0) + q->bits) {
+      case 8 + 2: s = run_tc<true, 1>(tmap, a, st); break;
+      case 8 + 3: s = run_tc<true, 2>(tmap, a, st); break;
+      case 8 + 4: s = run_tc<true, 3>(tmap, a, st); break;
+      case 1: s = run_tc<false, 1>(tmap, a, st); break;
+      case 2: s = run_tc<false, 2>(tmap, a, st); break;
+      case 3: s = run_tc<false, 3>(tmap, a, st); break;
+      case 4: s = run_tc<false, 4>(tmap, a, st); break;
       default: s = TQ_EUNSUPPORTED;
     }
     if (s != TQ_OK) return s;
   }
   return TQ_OK;
+}
+
+namespace {
+// One thread waits on an mbarrier phase that nothing completes and gives up after limit_ns:
+// the bounded-wait error path, without a device fault.
+__global__ void k_selftest_wait(uint64_t limit_ns, int* err) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    if (!mbar_wait_ns(&bar, 0, limit_ns)) atomicOr(err, 1);
+  }
+}
+}  // namespace
+
+tq_status launch_selftest_wait(uint32_t limit_us, cudaStream_t st) {
+  int* err = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_tq_device_error) != cudaSuccess)
+    return TQ_ECUDA;
+  k_selftest_wait<<<1, 32, 0, st>>>(static_cast<uint64_t>(limit_us) * 1000ull, err);
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ECUDA;
 }
 
 tq_status take_device_error(cudaStream_t st) {

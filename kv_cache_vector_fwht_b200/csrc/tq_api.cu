@@ -75,6 +75,11 @@ tq_status tq_sync_status(void* stream) {
   return take_device_error(static_cast<cudaStream_t>(stream));
 }
 
+tq_status tq_selftest_bounded_wait(uint32_t limit_us, void* stream) {
+  if (limit_us == 0 || limit_us > 2000000u) return TQ_EINVAL;
+  return launch_selftest_wait(limit_us, static_cast<cudaStream_t>(stream));
+}
+
 const char* tq_status_string(tq_status s) {
   switch (s) {
     case TQ_OK: return "ok";

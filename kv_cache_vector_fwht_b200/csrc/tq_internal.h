@@ -84,6 +84,8 @@ tq_status launch_keys_tc(const tq_quantizer* q, const void* x, int64_t n_rows, i
                          tq_key_planes out, RowMap map, cudaStream_t st);
 // Synchronise `st`; TQ_ETIMEOUT (and clear the flag) if a kernel gave up a bounded wait.
 tq_status take_device_error(cudaStream_t st);
+// A one-thread kernel whose bounded mbarrier wait runs out (sets the error flag).
+tq_status launch_selftest_wait(uint32_t limit_us, cudaStream_t st);
 
 // Fused append of a few tokens (mse / prod keys + values + lengths in one launch).
 constexpr int kMaxAppendBatch = 64;

@@ -96,3 +96,10 @@ def test_workspace_size_is_host_only():
     assert tq._lib.tq_decode_workspace_bytes(ctypes.byref(desc), 28, ctypes.byref(n)) == 0
     assert n.value > 8 * 28 * 132 * 4
     assert tq._lib.tq_decode_workspace_bytes(ctypes.byref(desc), 0, ctypes.byref(n)) == tq.TQ_EINVAL
+
+
+@pytest.mark.parametrize("limit_us", [0, 2_000_001])
+def test_selftest_wait_limit_checked_on_host(limit_us):
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_selftest_bounded_wait(limit_us)
+    assert e.value.status == tq.TQ_EINVAL
