@@ -85,13 +85,14 @@ __device__ __forceinline__ uint64_t sign_pair(int mask) {
 }
 
 // Shared-memory plan.
-template <int MB, int VB>
+template <int MB, int VB, bool PROD>
 struct Lay {
   static constexpr int IB = kD * storage_width_c(MB) / 8;  // index bytes per token
   static constexpr int PI = IB;                            // index positions (bytes)
   static constexpr int EI = MB == 3 ? 32 : 128;            // canonical entries per position
-  static constexpr int PS = 16;                            // sign positions
+  static constexpr int PS = PROD ? 16 : 0;                 // sign positions (prod only)
   static constexpr int ES = 128;
+  static constexpr int NB = PROD ? 4 : 2;                  // norm bytes per token
   static constexpr int VQB = VB ? kD * VB / 8 : 0;         // value code bytes per token
   static constexpr int VPB = VB ? 16 : 0;                  // value params per token
   static constexpr int lutI = 0;
@@ -116,6 +117,7 @@ struct Lay {
   static constexpr int scratch_bytes = (2 * 16 * (MB == 3 ? 0 : PI) + 2 * 16 * PS) * 16;
   static constexpr int total = (end_v - wv) >= merge ? end_v : wv + merge;
   static_assert(scratch + scratch_bytes <= total, "prologue scratch fits");
+  static_assert(total <= 227 * 1024, "decode shared memory budget");
 };
 
 // Accumulate one 4-head table entry with sign: acc[j] += sg * entry.
@@ -160,9 +162,11 @@ __device__ __forceinline__ void block_lookups(uint64_t (&acc)[2], uint32_t R0, u
   }
 }
 
-template <int MB, int VB, int NH>
+// PROD: prod keys (indices of MB = bits - 1, QJL signs, two norms); else mse keys (MB = bits,
+// one norm): s = n16 <Pi q, c[idx]>.
+template <int MB, int VB, int NH, bool PROD>
 __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ DecodeArgs a) {
-  using Lo = Lay<MB, VB>;
+  using Lo = Lay<MB, VB, PROD>;
   constexpr int IB = Lo::IB, PI = Lo::PI;
   static_assert(NH >= 1 && NH <= kMaxHeads, "heads per CTA");
   constexpr bool HAS_V = VB != 0;
@@ -205,11 +209,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     {
       const int tp1 = min(a.max_len, t0 + a.tokens_per_split);
       const int n = tp1 - t0;
-      const uint8_t* rng[5] = {a.k_idx + (kvrow + t0) * Lay<MB, VB>::IB, a.k_sgn + (kvrow + t0) * 16,
-                               reinterpret_cast<const uint8_t*>(a.k_nrm) + (kvrow + t0) * 4,
-                               a.v_q + (kvrow + t0) * Lay<MB, VB>::VQB,
+      const uint8_t* rng[5] = {a.k_idx + (kvrow + t0) * Lo::IB, a.k_sgn + (kvrow + t0) * 16,
+                               reinterpret_cast<const uint8_t*>(a.k_nrm) + (kvrow + t0) * Lo::NB,
+                               a.v_q + (kvrow + t0) * Lo::VQB,
                                reinterpret_cast<const uint8_t*>(a.v_par) + (kvrow + t0) * 16};
-      const int len_b[5] = {n * Lay<MB, VB>::IB, n * 16, n * 4, n * Lay<MB, VB>::VQB, VB ? n * 16 : 0};
+      const int len_b[5] = {n * Lo::IB, PROD ? n * 16 : 0, n * Lo::NB, n * Lo::VQB, VB ? n * 16 : 0};
 #pragma unroll
       for (int r = 0; r < 5; ++r)
         for (int off = threadIdx.x * 128; off < len_b[r]; off += kThreads * 128)
@@ -226,9 +230,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
           const uint4 v = __ldg(ip + i);
           iw[4 * i] = v.x; iw[4 * i + 1] = v.y; iw[4 * i + 2] = v.z; iw[4 * i + 3] = v.w;
         }
-        const uint4 s4 = __ldg(reinterpret_cast<const uint4*>(a.k_sgn + (kvrow + t) * 16));
-        sg[0] = s4.x; sg[1] = s4.y; sg[2] = s4.z; sg[3] = s4.w;
-        nn = __ldg(reinterpret_cast<const uint32_t*>(a.k_nrm) + kvrow + t);
+        if constexpr (PROD) {
+          const uint4 s4 = __ldg(reinterpret_cast<const uint4*>(a.k_sgn + (kvrow + t) * 16));
+          sg[0] = s4.x; sg[1] = s4.y; sg[2] = s4.z; sg[3] = s4.w;
+          nn = __ldg(reinterpret_cast<const uint32_t*>(a.k_nrm) + kvrow + t);
+        } else {
+          sg[0] = sg[1] = sg[2] = sg[3] = 0u;
+          nn = __ldg(a.k_nrm + kvrow + t);
+        }
       } else {
 #pragma unroll
         for (int i = 0; i < IB / 4; ++i) iw[i] = 0u;
@@ -255,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     const DevTables* __restrict__ tab = a.tab;
     // S_rot rows [16 warp, 16 warp + 16) as mma.sync A fragments (warps 0..7), from L2
     uint32_t afr[8][4];
-    if (warp < 8) {
+    if (PROD && warp < 8) {
       const int g = lane >> 2, t = lane & 3;
       const uint32_t* r0 = reinterpret_cast<const uint32_t*>(tab->s_rot + (16 * warp + g) * kD);
       const uint32_t* r1 = r0 + 8 * kD / 2;
@@ -310,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     }
     if (threadIdx.x < 16) sCen[threadIdx.x] = tab->cent[0][threadIdx.x];
     __syncthreads();
-    if (warp < 8) {
+    if (PROD && warp < 8) {
       // Sq = S_rot q_rot / sqrt(d) for the head slots on tensor cores: mma.sync m16n8k16
       // (fp16 S_rot is exact; q_rot enters as hi + lo fp16 halves; fp32 accumulation).
       const int g = lane >> 2, t = lane & 3;
@@ -357,9 +366,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
       // scratch region first; entry (e, p) = N[0][e mod 16][p] + N[1][e / 16][p].
       float4* NI = reinterpret_cast<float4*>(smem + Lo::scratch);
       float4* NS = NI + (MB == 3 ? 0 : 2 * 16 * PI);
-      constexpr int PN = MB == 2 ? PI : (MB == 1 ? PI : 0);  // nibble positions = byte positions
+      constexpr int PN = MB == 3 ? 0 : PI;  // nibble positions = byte positions
       if constexpr (MB != 3) {
-        constexpr int CPN = MB == 2 ? 2 : 4;  // coordinates per nibble
+        constexpr int CPN = 4 / MB;  // coordinates per nibble (MB = 1, 2 or 4)
         for (int i = threadIdx.x; i < 2 * 16 * PN; i += kThreads) {
           const int pp = i % PN, n = (i / PN) % 16, hf = i / (16 * PN);
           float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -434,11 +443,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
       const bool valid = lane < wcount;
 
       uint64_t accI[2] = {0ull, 0ull}, accS[2] = {0ull, 0ull};
+      if constexpr (PROD) {
 #pragma unroll
-      for (int blk = 0; blk < 2; ++blk) {
-        uint32_t R0, R1;
-        rot_block(sw4[2 * blk], sw4[2 * blk + 1], swap, sh, R0, R1);
-        block_lookups<Lo::PS * 16>(accS, R0, R1, lutS, blk, rot16);
+        for (int blk = 0; blk < 2; ++blk) {
+          uint32_t R0, R1;
+          rot_block(sw4[2 * blk], sw4[2 * blk + 1], swap, sh, R0, R1);
+          block_lookups<Lo::PS * 16>(accS, R0, R1, lutS, blk, rot16);
+        }
       }
       if constexpr (MB != 3) {
 #pragma unroll
@@ -463,13 +474,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
           }
         }
       }
-      const float n16 = half_lo(nw), r16 = half_hi(nw);
+      const float n16 = half_lo(nw), r16 = PROD ? half_hi(nw) : 0.f;
       float sc[kMaxHeads];
 #pragma unroll
       for (int j = 0; j < kMaxHeads / 2; ++j) {
         const float2 xi = up2(accI[j]), xs = up2(accS[j]);
-        sc[2 * j] = fmaf(n16, xi.x, r16 * xs.x);
-        sc[2 * j + 1] = fmaf(n16, xi.y, r16 * xs.y);
+        sc[2 * j] = PROD ? fmaf(n16, xi.x, r16 * xs.x) : n16 * xi.x;
+        sc[2 * j + 1] = PROD ? fmaf(n16, xi.y, r16 * xs.y) : n16 * xi.y;
       }
       if (a.scores != nullptr && valid) {
 #pragma unroll
@@ -734,11 +745,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
   if (threadIdx.x == 0) a.counters[static_cast<int64_t>(b) * a.n_q_heads + a.g_heads[grp][0]] = 0;
 }
 
-template <int MB, int VB, int NH>
+template <int MB, int VB, int NH, bool PROD>
 tq_status run_decode(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
-  constexpr int smem = Lay<MB, VB>::total;
-  static_assert(smem <= 227 * 1024, "decode shared memory budget");
-  auto kern = k_decode<MB, VB, NH>;
+  constexpr int smem = Lay<MB, VB, PROD>::total;
+  auto kern = k_decode<MB, VB, NH, PROD>;
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
@@ -760,11 +770,11 @@ tq_status run_decode(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ECUDA;
 }
 
-template <int MB, int VB>
+template <int MB, int VB, bool PROD>
 tq_status run_decode_nh(const DecodeArgs& a, dim3 grid, int max_heads, cudaStream_t st) {
-  if (max_heads <= 2) return run_decode<MB, VB, 2>(a, grid, st);
-  if (max_heads == 3) return run_decode<MB, VB, 3>(a, grid, st);
-  return run_decode<MB, VB, 4>(a, grid, st);
+  if (max_heads <= 2) return run_decode<MB, VB, 2, PROD>(a, grid, st);
+  if (max_heads == 3) return run_decode<MB, VB, 3, PROD>(a, grid, st);
+  return run_decode<MB, VB, 4, PROD>(a, grid, st);
 }
 
 int max_splits_for(int capacity) {
@@ -862,18 +872,31 @@ tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* c, const void*
   a.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + ((parts + 255) / 256) * 256);
 
   const dim3 grid(a.n_splits, n_groups, c->batch);
-  const int mb = q->bits - 1;
+  const bool prod = q->mode == TQ_MODE_PROD;
+  const int mb = prod ? q->bits - 1 : q->bits;
   const int vb = c->value_bits;
-  switch (mb * 8 + vb) {
-    case 1 * 8 + 0: return run_decode_nh<1, 0>(a, grid, max_heads, st);
-    case 1 * 8 + 2: return run_decode_nh<1, 2>(a, grid, max_heads, st);
-    case 1 * 8 + 4: return run_decode_nh<1, 4>(a, grid, max_heads, st);
-    case 2 * 8 + 0: return run_decode_nh<2, 0>(a, grid, max_heads, st);
-    case 2 * 8 + 2: return run_decode_nh<2, 2>(a, grid, max_heads, st);
-    case 2 * 8 + 4: return run_decode_nh<2, 4>(a, grid, max_heads, st);
-    case 3 * 8 + 0: return run_decode_nh<3, 0>(a, grid, max_heads, st);
-    case 3 * 8 + 2: return run_decode_nh<3, 2>(a, grid, max_heads, st);
-    case 3 * 8 + 4: return run_decode_nh<3, 4>(a, grid, max_heads, st);
+  switch ((prod ? 64 : 0) + mb * 8 + vb) {
+    case 64 + 1 * 8 + 0: return run_decode_nh<1, 0, true>(a, grid, max_heads, st);
+    case 64 + 1 * 8 + 2: return run_decode_nh<1, 2, true>(a, grid, max_heads, st);
+    case 64 + 1 * 8 + 4: return run_decode_nh<1, 4, true>(a, grid, max_heads, st);
+    case 64 + 2 * 8 + 0: return run_decode_nh<2, 0, true>(a, grid, max_heads, st);
+    case 64 + 2 * 8 + 2: return run_decode_nh<2, 2, true>(a, grid, max_heads, st);
+    case 64 + 2 * 8 + 4: return run_decode_nh<2, 4, true>(a, grid, max_heads, st);
+    case 64 + 3 * 8 + 0: return run_decode_nh<3, 0, true>(a, grid, max_heads, st);
+    case 64 + 3 * 8 + 2: return run_decode_nh<3, 2, true>(a, grid, max_heads, st);
+    case 64 + 3 * 8 + 4: return run_decode_nh<3, 4, true>(a, grid, max_heads, st);
+    case 1 * 8 + 0: return run_decode_nh<1, 0, false>(a, grid, max_heads, st);
+    case 1 * 8 + 2: return run_decode_nh<1, 2, false>(a, grid, max_heads, st);
+    case 1 * 8 + 4: return run_decode_nh<1, 4, false>(a, grid, max_heads, st);
+    case 2 * 8 + 0: return run_decode_nh<2, 0, false>(a, grid, max_heads, st);
+    case 2 * 8 + 2: return run_decode_nh<2, 2, false>(a, grid, max_heads, st);
+    case 2 * 8 + 4: return run_decode_nh<2, 4, false>(a, grid, max_heads, st);
+    case 3 * 8 + 0: return run_decode_nh<3, 0, false>(a, grid, max_heads, st);
+    case 3 * 8 + 2: return run_decode_nh<3, 2, false>(a, grid, max_heads, st);
+    case 3 * 8 + 4: return run_decode_nh<3, 4, false>(a, grid, max_heads, st);
+    case 4 * 8 + 0: return run_decode_nh<4, 0, false>(a, grid, max_heads, st);
+    case 4 * 8 + 2: return run_decode_nh<4, 2, false>(a, grid, max_heads, st);
+    case 4 * 8 + 4: return run_decode_nh<4, 4, false>(a, grid, max_heads, st);
     default: return TQ_EUNSUPPORTED;
   }
 }

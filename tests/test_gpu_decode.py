@@ -32,14 +32,14 @@ def run_decode(qg, cache, Q, q_dtype, out_dtype, head_map=None, sm_scale=0.0, sc
             scores.cpu().numpy() if scores is not None else None, ws)
 
 
-def small_case(seed, B, Hq, Hkv, lengths, cap, bits, vbits):
+def small_case(seed, B, Hq, Hkv, lengths, cap, bits, vbits, mode="prod"):
     g = W.rng(seed)
     N = max(lengths)
     K = W.round_bf16(W.scaled_gaussian_rows(g, B * Hkv * N).reshape(B, Hkv, N, 128))
     V = W.round_bf16(W.gaussian(g, (B, Hkv, N, 128)))
     Q = W.round_bf16(W.gaussian(g, (B, Hq, 128)))
-    qo = O.build_quantizer(128, bits, "prod", seed)
-    qg = tq.tq_build_codebook(128, bits, "prod", seed)
+    qo = O.build_quantizer(128, bits, mode, seed)
+    qg = tq.tq_build_codebook(128, bits, mode, seed)
     oc = oracle_cache(qo, K, V if vbits else None, vbits, lengths)
     cache = tq.KVCache(qg, B, Hkv, cap, value_bits=vbits, device="cuda:0")
     upload_cache(cache, oc)
@@ -59,6 +59,29 @@ def test_decode_small_ragged(bits, vbits, q_dtype, out_dtype):
     ref, _ = O.decode_attention(qo, oc, Q.astype(np.float64), value_bits=vbits)
     err = check_attention(out, ref, out_dtype == torch.bfloat16)
     print(bits, vbits, err)
+
+
+@pytest.mark.parametrize("bits,vbits", [(1, 2), (2, 2), (3, 4), (4, 4), (4, 2)])
+def test_decode_mse_keys(bits, vbits):
+    """mse caches: s = n16 <Pi q, c[idx]> (no QJL term), 1..4-bit indices."""
+    require_cuda()
+    qo, qg, oc, cache, Q = small_case(60 + bits, 2, 7, 2, [1100, 613], 1152, bits, vbits, "mse")
+    hm = [0, 0, 0, 0, 1, 1, 1]   # groups of 4 and 3 query heads
+    out, _, _ = run_decode(qg, cache, Q, torch.bfloat16, torch.float32, head_map=hm)
+    ref, _ = O.decode_attention(qo, oc, Q.astype(np.float64), head_map=hm, value_bits=vbits)
+    err = check_attention(out, ref, False)
+    print("mse", bits, vbits, err)
+
+
+@pytest.mark.parametrize("bits", [1, 3, 4])
+def test_decode_mse_scores(bits):
+    require_cuda()
+    qo, qg, oc, cache, Q = small_case(70 + bits, 1, 8, 1, [777], 784, bits, 0, "mse")
+    _, sc, _ = run_decode(qg, cache, Q, torch.float32, torch.float32, scores_ld=784)
+    _, ref = O.decode_attention(qo, oc, Q.astype(np.float64), value_bits=0, want_scores=True)
+    for h in range(8):
+        check_scores(sc[0, h, :777], ref[0][h], np.linalg.norm(Q[0, h]),
+                     O.fp16_from_bits(oc["k_norms"][0, 0, :777, 0]))
 
 
 def test_decode_head_map_scale_and_scores():
