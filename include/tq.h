@@ -154,6 +154,17 @@ tq_status tq_host_tables(int d, int bits, int mode, uint64_t seed,
 tq_status tq_quantize_keys(const tq_quantizer* q, const void* x_dev, int dtype,
                            int64_t n_rows, int64_t ld, tq_key_planes out, void* stream);
 
+/* Dequantize n_rows packed keys (`planes`, the layout tq_quantize_keys writes) into out_dev
+ * (n_rows x ld, TQ_F32 or TQ_BF16, same row rules as tq_quantize_keys' input), in the
+ * original coordinates (validate_paper.py dequantize; tqlite prod.py):
+ *   mse:     x_hat = ||x|| Pi^T c[idx]
+ *   prod:    x_hat = ||x|| Pi^T c[idx] + ||r|| sqrt(pi/2)/d S^T (2 sigma - 1)   (S = S_rot Pi),
+ *            so that <q, x_hat> equals the decode estimator s(q)
+ *   grouped: each group's mse reconstruction on its own channels.
+ * n_rows = 0 is a no-op. Not part of the decode hot path (quality checks, debugging). */
+tq_status tq_dequantize_keys(const tq_quantizer* q, tq_key_planes planes, int64_t n_rows,
+                             void* out_dev, int out_dtype, int64_t ld, void* stream);
+
 /* Quantize n_rows value vectors v_dev (n_rows x ld, TQ_F32 or TQ_BF16; d = 128) into
  * `out`: per group of `group` (= 32) channels, mn = min, scale = (max - mn)/(2^bits - 1),
  * stored as fp16; code = clamp(rint((v - mn16)/s16), 0, 2^bits - 1), 0 if s16 = 0; the
@@ -182,7 +193,7 @@ tq_status tq_decode_workspace_bytes(const tq_kv_cache* cache, int n_q_heads, siz
  *   out = softmax(sm_scale * s) . v_hat,   v_hat = mn16 + code * s16.
  * The kernel is launched with programmatic dependent launch: after tq_append on the same
  * stream its query-only prologue overlaps the append kernel; it reads the lengths and the
- * cache only once the preceding kernels have completed. */
+ * cache only once the preceding kernels have completed.
  * q_dev: batch x n_q_heads x d (TQ_F32 or TQ_BF16). head_map: host int32[n_q_heads] with
  * values in [0, n_kv_heads), NULL = h / (n_q_heads / n_kv_heads). sm_scale <= 0 means
  * 1/sqrt(d). out_dev: batch x n_q_heads x d in out_dtype (TQ_F32 or TQ_BF16), may be NULL

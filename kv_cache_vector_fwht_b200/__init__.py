@@ -28,7 +28,7 @@ TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 D = 128
 
 EXPORTED = ["tq_build_codebook", "tq_free", "tq_key_layout", "tq_host_tables",
-            "tq_quantize_keys", "tq_quantize_values", "tq_append", "tq_decode_workspace_bytes",
+            "tq_quantize_keys", "tq_dequantize_keys", "tq_quantize_values", "tq_append", "tq_decode_workspace_bytes",
             "tq_decode_attention", "tq_decode_attention_noalloc", "tq_sync_status",
             "tq_selftest_bounded_wait", "tq_status_string", "tq_abi_version"]
 
@@ -67,6 +67,9 @@ _lib.tq_host_tables.restype = c_int
 _lib.tq_quantize_keys.argtypes = [c_void_p, c_void_p, c_int, c_int64, c_int64, KeyPlanes,
                                   c_void_p]
 _lib.tq_quantize_keys.restype = c_int
+_lib.tq_dequantize_keys.argtypes = [c_void_p, KeyPlanes, c_int64, c_void_p, c_int, c_int64,
+                                    c_void_p]
+_lib.tq_dequantize_keys.restype = c_int
 _lib.tq_quantize_values.argtypes = [c_void_p, c_int, c_int64, c_int64, c_int, c_int, c_int,
                                     ValuePlanes, c_void_p]
 _lib.tq_quantize_values.restype = c_int
@@ -223,6 +226,14 @@ def tq_quantize_keys(q: Quantizer, x, planes: dict, stream=None) -> None:
     assert x.dim() == 2 and x.stride(1) == 1
     _check(_lib.tq_quantize_keys(q.handle, _ptr(x), _dtype_code(x), x.shape[0], x.stride(0),
                                  _key_planes(planes), _stream(stream)), "tq_quantize_keys")
+
+
+def tq_dequantize_keys(q: Quantizer, planes: dict, out, stream=None) -> None:
+    """planes: key planes of out.shape[0] rows; out: (n_rows, ld>=128) fp32/bf16 CUDA tensor."""
+    assert out.dim() == 2 and out.stride(1) == 1
+    _check(_lib.tq_dequantize_keys(q.handle, _key_planes(planes), out.shape[0],
+                                   _ptr(out), _dtype_code(out), out.stride(0), _stream(stream)),
+           "tq_dequantize_keys")
 
 
 def alloc_value_planes(n_rows: int, bits: int, d: int = D, group: int = 32, device="cuda"):

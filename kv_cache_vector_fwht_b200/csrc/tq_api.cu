@@ -210,6 +210,17 @@ tq_status tq_quantize_keys(const tq_quantizer* q, const void* x, int dtype, int6
                               static_cast<cudaStream_t>(stream));
 }
 
+tq_status tq_dequantize_keys(const tq_quantizer* q, tq_key_planes planes, int64_t n_rows,
+                             void* out, int out_dtype, int64_t ld, void* stream) {
+  if (!q) return TQ_EINVAL;
+  tq_status st = check_rows(out, out_dtype, n_rows, ld);
+  if (st != TQ_OK) return st;
+  if (n_rows == 0) return TQ_OK;
+  if ((st = check_key_planes(q, planes)) != TQ_OK) return st;
+  return launch_dequantize_keys(q, planes, n_rows, out, out_dtype, ld,
+                                static_cast<cudaStream_t>(stream));
+}
+
 tq_status tq_quantize_values(const void* v, int dtype, int64_t n_rows, int64_t ld, int d, int bits,
                              int group, tq_value_planes out, void* stream) {
   if (d != kD) return TQ_EUNSUPPORTED;

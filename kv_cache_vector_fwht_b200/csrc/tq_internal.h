@@ -78,6 +78,9 @@ tq_status launch_quantize_keys(const tq_quantizer* q, const void* x, int dtype, 
 tq_status launch_quantize_values(const void* v, int dtype, int64_t n_rows, int64_t ld, int bits,
                                  tq_value_planes out, RowMap map, cudaStream_t st);
 tq_status launch_advance_len(int32_t* len, int batch, int n, cudaStream_t st);
+// packed key planes back to vectors in the original coordinates
+tq_status launch_dequantize_keys(const tq_quantizer* q, tq_key_planes planes, int64_t n_rows,
+                                 void* out, int out_dtype, int64_t ld, cudaStream_t st);
 // prod-mode bf16 keys with the QJL projection on tcgen05 tensor cores
 bool keys_tc_ok(const tq_quantizer* q, int dtype);
 tq_status launch_keys_tc(const tq_quantizer* q, const void* x, int64_t n_rows, int64_t ld,

@@ -101,3 +101,50 @@ def test_append_key_only_cache_and_errors():
     assert e.value.status == tq.TQ_EINVAL
     with pytest.raises(ValueError):
         tq.KVCache(qg, 1, 1, 20, device=dev)
+
+
+@pytest.mark.parametrize("mode,bits,vbits,dtype", [("prod", 3, 2, torch.bfloat16),
+                                                   ("prod", 2, 4, torch.float32),
+                                                   ("mse", 4, 2, torch.bfloat16),
+                                                   ("grouped", 3, 2, torch.bfloat16)])
+def test_append_multi_token_chunks(mode, bits, vbits, dtype):
+    """Prefill in ragged chunks (store.py append_chunk): chunk sizes on both sides of the
+    64-token switch between the fused append kernel and the separate quantize kernels, ragged
+    starting lengths, bf16 and fp32 inputs. Every cached row matches the oracle's quantization
+    of the whole prefix, so chunk boundaries leave no trace."""
+    dev = require_cuda()
+    ch = W.outlier_channels(6)
+    outl = ch if mode == "grouped" else None
+    qg = tq.tq_build_codebook(128, bits, mode, 8, outl)
+    qo = O.build_quantizer(128, bits, mode, 8, outl)
+    B, H, cap = 2, 3, 544
+    start = [0, 17]
+    chunks = [1, 63, 64, 65, 130, 200]
+    total = sum(chunks)
+    cache = tq.KVCache(qg, B, H, cap, value_bits=vbits, device=dev)
+    cache.set_lengths(start)
+    g = W.rng(77)
+    k = W.scaled_gaussian_rows(g, B * H * total).reshape(B, H, total, 128)
+    if dtype == torch.bfloat16:
+        k = W.round_bf16(k)
+    v = W.gaussian(g, (B, H, total, 128))
+    v = W.round_bf16(v) if dtype == torch.bfloat16 else v.astype(np.float32).astype(np.float64)
+    k = k if dtype == torch.bfloat16 else k.astype(np.float32).astype(np.float64)
+    t0 = 0
+    for n_tok in chunks:
+        tq.tq_append(qg, cache, to_device(k[:, :, t0:t0 + n_tok], dtype).contiguous(),
+                     to_device(v[:, :, t0:t0 + n_tok], dtype).contiguous())
+        t0 += n_tok
+    torch.cuda.synchronize()
+    assert cache.lengths == [s + total for s in start]
+    assert cache.len_dev.cpu().tolist() == cache.lengths
+    for b in range(B):
+        for h in range(H):
+            base = (b * H + h) * cap + start[b]
+            rows = slice(base, base + total)
+            gp = to_np_planes({"idx": cache.k_idx[rows], "signs": None if cache.k_signs is None
+                               else cache.k_signs[rows], "norms": cache.k_norms[rows]})
+            check_key_parity(qo, k[b, h].astype(np.float64), gp)
+            ref = O.quantize_values(v[b, h].astype(np.float64), vbits)
+            assert np.array_equal(cache.v_q[rows].cpu().numpy(), ref["q"])
+            assert np.array_equal(cache.v_params[rows].cpu().numpy().view(np.uint16), ref["params"])
