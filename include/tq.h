@@ -186,10 +186,11 @@ tq_status tq_append(const tq_quantizer* q, tq_kv_cache* cache, const void* k_new
  * workspace must be zero-filled before its first use; every call leaves it reusable. */
 tq_status tq_decode_workspace_bytes(const tq_kv_cache* cache, int n_q_heads, size_t* bytes);
 
-/* Fused decode attention over a packed prod- or mse-mode cache (grouped: TQ_EUNSUPPORTED),
- * one query token per sequence. For query head h of sequence b with KV head kv = head_map[h]:
- *   prod: s_i = ||x_i|| <Pi q, c[idx_i]> + ||r_i|| sqrt(pi/2)/d <S q, 2 sigma_i - 1>
- *   mse:  s_i = ||x_i|| <Pi q, c[idx_i]>                                          (i < len[b])
+/* Fused decode attention over a packed cache of any key mode, one query token per sequence.
+ * For query head h of sequence b with KV head kv = head_map[h], and every i < len[b]:
+ *   prod:    s_i = ||x_i|| <Pi q, c[idx_i]> + ||r_i|| sqrt(pi/2)/d <S q, 2 sigma_i - 1>
+ *   mse:     s_i = ||x_i|| <Pi q, c[idx_i]>
+ *   grouped: s_i = sum over the two channel groups g of ||x_i,g|| <Pi_g q_g, c_g[idx_i,g]>
  *   out = softmax(sm_scale * s) . v_hat,   v_hat = mn16 + code * s16.
  * The kernel is launched with programmatic dependent launch: after tq_append on the same
  * stream its query-only prologue overlaps the append kernel; it reads the lengths and the

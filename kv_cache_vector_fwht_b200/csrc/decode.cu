@@ -1,4 +1,4 @@
-// Fused decode attention over a packed prod-mode KV cache (sm_100a).
+// Fused decode attention over a packed KV cache: prod, mse or grouped keys (sm_100a).
 //
 // Estimator (Implementing TurboQuant (part 5), algorithm overview; validate_paper.py
 // attention_score):  s_i = n16_i <Pi q, c[idx_i]> + r16_i sqrt(pi/2)/d <S q, 2 sigma_i - 1>.
@@ -84,15 +84,28 @@ __device__ __forceinline__ uint64_t sign_pair(int mask) {
   return pk2(s, s);
 }
 
-// Shared-memory plan.
-template <int MB, int VB, bool PROD>
+// Key kinds: mse (indices, one norm), prod (indices + QJL signs, two norms), grouped (a
+// 32-channel outlier group at b + 1 bits and a 96-channel group at b bits, one norm each).
+enum KeyKind { kMse = 0, kProd = 1, kGrp = 2 };
+
+// Shared-memory plan. MB: index bits (mse, prod) or the grouped base bits b. A token's key
+// bytes form two lookup segments: I (index bytes; grouped: the outlier group) and S (prod:
+// the QJL sign bytes; grouped: the normal group, padded with zero bytes to whole 8-byte
+// blocks). Each segment accumulates its own sum; the two norms scale them.
+template <int MB, int VB, int K>
 struct Lay {
-  static constexpr int IB = kD * storage_width_c(MB) / 8;  // index bytes per token
-  static constexpr int PI = IB;                            // index positions (bytes)
-  static constexpr int EI = MB == 3 ? 32 : 128;            // canonical entries per position
-  static constexpr int PS = PROD ? 16 : 0;                 // sign positions (prod only)
-  static constexpr int ES = 128;
-  static constexpr int NB = PROD ? 4 : 2;                  // norm bytes per token
+  static constexpr bool GRP = K == kGrp;
+  static constexpr int MI = GRP ? MB + 1 : MB;                     // segment I code bits
+  static constexpr int MS = GRP ? MB : 1;                          // segment S code bits
+  static constexpr int IBI = (GRP ? 32 : kD) * storage_width_c(MI) / 8;
+  static constexpr int IBS = GRP ? 96 * storage_width_c(MS) / 8 : 0;
+  static constexpr int IB = IBI + IBS;                             // index-plane bytes per token
+  static constexpr int PI = IBI;                                   // segment I positions
+  static constexpr int EI = MI == 3 ? 32 : 128;                    // canonical entries per position
+  static constexpr int PS = K == kProd ? 16 : (GRP ? (IBS + 7) / 8 * 8 : 0);
+  static constexpr int ES = MS == 3 ? 32 : 128;
+  static constexpr int KW = (IBI + (GRP ? PS : 0)) / 4;            // key words held per token
+  static constexpr int NB = K == kMse ? 2 : 4;                     // norm bytes per token
   static constexpr int VQB = VB ? kD * VB / 8 : 0;         // value code bytes per token
   static constexpr int VPB = VB ? 16 : 0;                  // value params per token
   static constexpr int lutI = 0;
@@ -113,9 +126,12 @@ struct Lay {
   static constexpr int end_v = vpair + (VB ? kWarps * 4 * kVpStride * 16 : 0);
   static constexpr int merge = kWarps * kMaxHeads * kPartStride * 4;   // reuses wv..
   // prologue scratch for the nibble partial tables (the value slots may be filling then)
+  static constexpr int PNI = MI == 3 ? 0 : PI;                         // nibble-built positions
+  static constexpr int PNS = MS == 3 ? 0 : PS;
   static constexpr int scratch = VB ? ppair : wv;
-  static constexpr int scratch_bytes = (2 * 16 * (MB == 3 ? 0 : PI) + 2 * 16 * PS) * 16;
+  static constexpr int scratch_bytes = (2 * 16 * PNI + 2 * 16 * PNS) * 16;
   static constexpr int total = (end_v - wv) >= merge ? end_v : wv + merge;
+  static_assert(IBI % 8 == 0 && PS % 8 == 0, "whole 8-byte lookup blocks");
   static_assert(scratch + scratch_bytes <= total, "prologue scratch fits");
   static_assert(total <= 227 * 1024, "decode shared memory budget");
 };
@@ -162,12 +178,45 @@ __device__ __forceinline__ void block_lookups(uint64_t (&acc)[2], uint32_t R0, u
   }
 }
 
-// PROD: prod keys (indices of MB = bits - 1, QJL signs, two norms); else mse keys (MB = bits,
-// one norm): s = n16 <Pi q, c[idx]>.
-template <int MB, int VB, int NH, bool PROD>
+// Lookups of one 8-byte block of bytes holding two 3-bit codes in their nibbles: the mirror
+// flips both codes (k -> 7 - k), chosen by bit 6 (high code >= 4); entry = low code + 8 (high
+// code mod 4).
+template <int ROWB>
+__device__ __forceinline__ void block_lookups3(uint64_t (&acc)[2], uint32_t R0, uint32_t R1,
+                                               const uint8_t* tab, int blk,
+                                               const uint32_t (&rot16)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t v = ((i < 4 ? R0 : R1) >> (8 * (i & 3))) & 0xffu;
+    const int msk = static_cast<int>(v << 25) >> 31;
+    const uint32_t vc = v ^ (static_cast<uint32_t>(msk) & 0x77u);
+    const uint32_t en = (vc & 7u) | ((vc >> 1) & 0x18u);
+    lut_acc(acc, tab + 128 * blk + en * ROWB + rot16[i], sign_pair(msk));
+  }
+}
+
+// Segment lookups over 8-byte blocks of words w (2 words a block).
+template <int MBITS, int NPOS>
+__device__ __forceinline__ void segment_lookups(uint64_t (&acc)[2], const uint32_t* w,
+                                                const uint8_t* tab, bool swap, uint32_t sh,
+                                                const uint32_t (&rot16)[8]) {
+#pragma unroll
+  for (int blk = 0; blk < NPOS / 8; ++blk) {
+    uint32_t R0, R1;
+    rot_block(w[2 * blk], w[2 * blk + 1], swap, sh, R0, R1);
+    if constexpr (MBITS == 3) block_lookups3<NPOS * 16>(acc, R0, R1, tab, blk, rot16);
+    else block_lookups<NPOS * 16>(acc, R0, R1, tab, blk, rot16);
+  }
+}
+
+// K = kMse: s = n16 <Pi q, c[idx]>; kProd: + r16 sqrt(pi/2)/d <S q, 2 sigma - 1>;
+// kGrp: s = n_o <Pi_o q_o, c_o[idx_o]> + n_n <Pi_n q_n, c_n[idx_n]> over the two channel
+// groups (Pi_g: 32-point Hadamard blocks after the group's signs).
+template <int MB, int VB, int NH, int K>
 __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ DecodeArgs a) {
-  using Lo = Lay<MB, VB, PROD>;
-  constexpr int IB = Lo::IB, PI = Lo::PI;
+  using Lo = Lay<MB, VB, K>;
+  constexpr bool PROD = K == kProd, GRP = K == kGrp, TWO = K != kMse;
+  constexpr int IB = Lo::IB, PI = Lo::PI, KW = Lo::KW;
   static_assert(NH >= 1 && NH <= kMaxHeads, "heads per CTA");
   constexpr bool HAS_V = VB != 0;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -179,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
   uint8_t* qlo = smem + Lo::qlo;
   float* qinv = reinterpret_cast<float*>(smem + Lo::qinv);
   __shared__ int sLast;
-  __shared__ float sCen[16];
+  __shared__ float sCen[32];
 
   const int split = blockIdx.x, grp = blockIdx.y, b = blockIdx.z;
   const int kv = a.g_kv[grp], nh = a.g_n[grp];
@@ -209,35 +258,49 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     {
       const int tp1 = min(a.max_len, t0 + a.tokens_per_split);
       const int n = tp1 - t0;
-      const uint8_t* rng[5] = {a.k_idx + (kvrow + t0) * Lo::IB, a.k_sgn + (kvrow + t0) * 16,
+      const uint8_t* rng[5] = {a.k_idx + (kvrow + t0) * IB, a.k_sgn + (kvrow + t0) * 16,
                                reinterpret_cast<const uint8_t*>(a.k_nrm) + (kvrow + t0) * Lo::NB,
                                a.v_q + (kvrow + t0) * Lo::VQB,
                                reinterpret_cast<const uint8_t*>(a.v_par) + (kvrow + t0) * 16};
-      const int len_b[5] = {n * Lo::IB, PROD ? n * 16 : 0, n * Lo::NB, n * Lo::VQB, VB ? n * 16 : 0};
+      const int len_b[5] = {n * IB, PROD ? n * 16 : 0, n * Lo::NB, n * Lo::VQB, VB ? n * 16 : 0};
 #pragma unroll
       for (int r = 0; r < 5; ++r)
         for (int off = threadIdx.x * 128; off < len_b[r]; off += kThreads * 128)
           asm volatile("prefetch.global.L2 [%0];" ::"l"(rng[r] + off));
     }
     // key bytes of this lane's token in chunk c (zeros past the range)
-    uint32_t kw[IB / 4], sw4[4], nw;
-    auto load_keys = [&](int ts, uint32_t (&iw)[IB / 4], uint32_t (&sg)[4], uint32_t& nn) {
+    // (grouped: the normal group's words are zero-padded to whole 8-byte blocks)
+    uint32_t kw[KW], sw4[4], nw;
+    auto load_keys = [&](int ts, uint32_t (&iw)[KW], uint32_t (&sg)[4], uint32_t& nn) {
       const int t = ts + lane;
-      if (t < t1) {
-        const uint4* ip = reinterpret_cast<const uint4*>(a.k_idx + (kvrow + t) * IB);
 #pragma unroll
-        for (int i = 0; i < IB / 16; ++i) {
-          const uint4 v = __ldg(ip + i);
-          iw[4 * i] = v.x; iw[4 * i + 1] = v.y; iw[4 * i + 2] = v.z; iw[4 * i + 3] = v.w;
+      for (int i = IB / 4; i < KW; ++i) iw[i] = 0u;
+      if (t < t1) {
+        const uint8_t* row = a.k_idx + (kvrow + t) * IB;
+        if constexpr (IB % 16 == 0) {
+#pragma unroll
+          for (int i = 0; i < IB / 16; ++i) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(row) + i);
+            iw[4 * i] = v.x; iw[4 * i + 1] = v.y; iw[4 * i + 2] = v.z; iw[4 * i + 3] = v.w;
+          }
+        } else if constexpr (IB % 8 == 0) {
+#pragma unroll
+          for (int i = 0; i < IB / 8; ++i) {
+            const uint2 v = __ldg(reinterpret_cast<const uint2*>(row) + i);
+            iw[2 * i] = v.x; iw[2 * i + 1] = v.y;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < IB / 4; ++i) iw[i] = __ldg(reinterpret_cast<const uint32_t*>(row) + i);
         }
         if constexpr (PROD) {
           const uint4 s4 = __ldg(reinterpret_cast<const uint4*>(a.k_sgn + (kvrow + t) * 16));
           sg[0] = s4.x; sg[1] = s4.y; sg[2] = s4.z; sg[3] = s4.w;
-          nn = __ldg(reinterpret_cast<const uint32_t*>(a.k_nrm) + kvrow + t);
         } else {
           sg[0] = sg[1] = sg[2] = sg[3] = 0u;
-          nn = __ldg(a.k_nrm + kvrow + t);
         }
+        if constexpr (TWO) nn = __ldg(reinterpret_cast<const uint32_t*>(a.k_nrm) + kvrow + t);
+        else nn = __ldg(a.k_nrm + kvrow + t);
       } else {
 #pragma unroll
         for (int i = 0; i < IB / 4; ++i) iw[i] = 0u;
@@ -283,14 +346,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
       if (warp < nh) {
         const int hq = a.g_heads[grp][warp];
         const int64_t qoff = (static_cast<int64_t>(b) * a.n_q_heads + hq) * kD;
-        if (a.q_f32) load4<true>(static_cast<const float*>(a.q) + qoff, 4 * lane, v);
-        else load4<false>(static_cast<const uint16_t*>(a.q) + qoff, 4 * lane, v);
+        if constexpr (GRP) {
+          // chain order: the outlier channels, then the normal channels
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int c = tab->chan[4 * lane + i];
+            v[i] = a.q_f32 ? static_cast<const float*>(a.q)[qoff + c]
+                           : __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t*>(a.q)[qoff + c]) << 16);
+          }
+        } else {
+          if (a.q_f32) load4<true>(static_cast<const float*>(a.q) + qoff, 4 * lane, v);
+          else load4<false>(static_cast<const uint16_t*>(a.q) + qoff, 4 * lane, v);
+        }
         const uint32_t sw = tab->sign_bits[lane >> 3];
 #pragma unroll
         for (int i = 0; i < 4; ++i) v[i] = flip_sign(v[i], sw, (4 * lane + i) & 31);
+        // 128-point transform; grouped: 32-point blocks (lanes 8k .. 8k + 7)
         fwht_reg<4>(v);
 #pragma unroll
-        for (int mm = 1; mm < 32; mm <<= 1) {
+        for (int mm = 1; mm < (GRP ? 8 : 32); mm <<= 1) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const float other = __shfl_xor_sync(kFull, v[i], mm);
@@ -317,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         reinterpret_cast<__half*>(qlo + warp * kSrotStride)[j] = lo;
       }
     }
-    if (threadIdx.x < 16) sCen[threadIdx.x] = tab->cent[0][threadIdx.x];
+    if (threadIdx.x < 32) sCen[threadIdx.x] = (&tab->cent[0][0])[threadIdx.x];
     __syncthreads();
     if (PROD && warp < 8) {
       // Sq = S_rot q_rot / sqrt(d) for the head slots on tensor cores: mma.sync m16n8k16
@@ -358,69 +432,86 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
       load_values(c0);
     }
     {
-      const float* cen = sCen;
-      const float cI = a.scale_log2 * (1.f / 128.f);
-      const float cS = a.scale_log2 * 1.2533141373155002512f / 128.f;  // sqrt(pi/2) / d
-      // Byte entries are sums of two nibble partials (low and high half of the byte):
-      // NI[half][n][p] and NS[half][n][p] (16-byte float4 of the 4 head slots) are built in a
-      // scratch region first; entry (e, p) = N[0][e mod 16][p] + N[1][e / 16][p].
+      constexpr int PNI = Lo::PNI, PNS = Lo::PNS, PS = Lo::PS;
+      const float* cenI = sCen;        // segment I centroids (grouped: the outlier group)
+      const float* cenS = sCen + 16;   // grouped: the normal group
+      // entry scales: 1/sqrt(d) of Pi times 1/sqrt(d) of the N(0,1)-scale centroids (grouped:
+      // 1/sqrt(32) of a Hadamard block times 1/sqrt(d_g)); prod signs: sqrt(pi/2)/d
+      const float cI = a.scale_log2 * (GRP ? 1.f / 32.f : 1.f / 128.f);
+      const float cS = GRP ? a.scale_log2 * 0.018042195912175807f
+                           : a.scale_log2 * 1.2533141373155002512f / 128.f;
+      // Entries of 1-, 2- and 4-bit code bytes and of sign bytes are sums of two nibble
+      // partials (low and high half of the byte): NI[half][n][p] and NS[half][n][p]
+      // (16-byte float4 of the 4 head slots) are built in a scratch region first; entry
+      // (e, p) = N[0][e mod 16][p] + N[1][e / 16][p].
       float4* NI = reinterpret_cast<float4*>(smem + Lo::scratch);
-      float4* NS = NI + (MB == 3 ? 0 : 2 * 16 * PI);
-      constexpr int PN = MB == 3 ? 0 : PI;  // nibble positions = byte positions
-      if constexpr (MB != 3) {
-        constexpr int CPN = 4 / MB;  // coordinates per nibble (MB = 1, 2 or 4)
-        for (int i = threadIdx.x; i < 2 * 16 * PN; i += kThreads) {
-          const int pp = i % PN, n = (i / PN) % 16, hf = i / (16 * PN);
+      float4* NS = NI + 2 * 16 * PNI;
+      if constexpr (PNI > 0) {
+        constexpr int CPN = 4 / Lo::MI;  // coordinates per nibble
+        for (int i = threadIdx.x; i < 2 * 16 * PNI; i += kThreads) {
+          const int pp = i % PNI, n = (i / PNI) % 16, hf = i / (16 * PNI);
           float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
           for (int f = 0; f < CPN; ++f) {
             const float4 x = *reinterpret_cast<const float4*>(qrT + (2 * CPN * pp + CPN * hf + f) * kMaxHeads);
-            const float c = cen[(n >> (MB * f)) & ((1 << MB) - 1)] * cI;
+            const float c = cenI[(n >> (Lo::MI * f)) & ((1 << Lo::MI) - 1)] * cI;
             r.x = fmaf(x.x, c, r.x); r.y = fmaf(x.y, c, r.y);
             r.z = fmaf(x.z, c, r.z); r.w = fmaf(x.w, c, r.w);
           }
-          NI[(hf * 16 + n) * PN + pp] = r;
+          NI[(hf * 16 + n) * PNI + pp] = r;
         }
       }
-      for (int i = threadIdx.x; i < 2 * 16 * Lo::PS; i += kThreads) {
-        const int pp = i % Lo::PS, n = (i / Lo::PS) % 16, hf = i / (16 * Lo::PS);
-        float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+      if constexpr (PNS > 0) {
+        for (int i = threadIdx.x; i < 2 * 16 * PNS; i += kThreads) {
+          const int pp = i % PNS, n = (i / PNS) % 16, hf = i / (16 * PNS);
+          float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+          if constexpr (PROD) {
 #pragma unroll
-        for (int f = 0; f < 4; ++f) {
-          const float4 x = *reinterpret_cast<const float4*>(sqT + (8 * pp + 4 * hf + f) * kMaxHeads);
-          const float sg = ((n >> f) & 1) ? cS : -cS;
-          r.x = fmaf(x.x, sg, r.x); r.y = fmaf(x.y, sg, r.y);
-          r.z = fmaf(x.z, sg, r.z); r.w = fmaf(x.w, sg, r.w);
+            for (int f = 0; f < 4; ++f) {
+              const float4 x = *reinterpret_cast<const float4*>(sqT + (8 * pp + 4 * hf + f) * kMaxHeads);
+              const float sg = ((n >> f) & 1) ? cS : -cS;
+              r.x = fmaf(x.x, sg, r.x); r.y = fmaf(x.y, sg, r.y);
+              r.z = fmaf(x.z, sg, r.z); r.w = fmaf(x.w, sg, r.w);
+            }
+          } else if (pp < Lo::IBS) {  // grouped normal group; padding positions stay zero
+            constexpr int CPN = 4 / Lo::MS;
+#pragma unroll
+            for (int f = 0; f < CPN; ++f) {
+              const float4 x = *reinterpret_cast<const float4*>(qrT + (32 + 2 * CPN * pp + CPN * hf + f) * kMaxHeads);
+              const float c = cenS[(n >> (Lo::MS * f)) & ((1 << Lo::MS) - 1)] * cS;
+              r.x = fmaf(x.x, c, r.x); r.y = fmaf(x.y, c, r.y);
+              r.z = fmaf(x.z, c, r.z); r.w = fmaf(x.w, c, r.w);
+            }
+          }
+          NS[(hf * 16 + n) * PNS + pp] = r;
         }
-        NS[(hf * 16 + n) * Lo::PS + pp] = r;
       }
       __syncthreads();
-      if constexpr (MB == 3) {
-        // byte = two 3-bit codes in nibbles: coords 2p, 2p+1 (entry e: codes e mod 8, e / 8)
-        constexpr int TPP = kThreads / PI;
-        const int p = threadIdx.x % PI, e0 = threadIdx.x / PI;
-        const float4 x = *reinterpret_cast<const float4*>(qrT + (2 * p) * kMaxHeads);
-        const float4 y = *reinterpret_cast<const float4*>(qrT + (2 * p + 1) * kMaxHeads);
-        for (int e = e0; e < Lo::EI; e += TPP) {
-          const float ca = cen[e & 7] * cI, cb = cen[e >> 3] * cI;
-          *reinterpret_cast<float4*>(lutI + (e * PI + p) * 16) =
+      // bytes of two 3-bit codes in nibbles: coordinates c0 + 2p, c0 + 2p + 1 (entry e: codes
+      // e mod 8 and e / 8)
+      auto build3 = [&](uint8_t* lut, int P, int c0, const float* cen, float cs) {
+        for (int i = threadIdx.x; i < 32 * P; i += kThreads) {
+          const int p = i % P, e = i / P;
+          const float4 x = *reinterpret_cast<const float4*>(qrT + (c0 + 2 * p) * kMaxHeads);
+          const float4 y = *reinterpret_cast<const float4*>(qrT + (c0 + 2 * p + 1) * kMaxHeads);
+          const float ca = cen[e & 7] * cs, cb = cen[e >> 3] * cs;
+          *reinterpret_cast<float4*>(lut + (e * P + p) * 16) =
               make_float4(fmaf(x.x, ca, y.x * cb), fmaf(x.y, ca, y.y * cb),
                           fmaf(x.z, ca, y.z * cb), fmaf(x.w, ca, y.w * cb));
         }
-      } else {
-        for (int i = threadIdx.x; i < Lo::EI * PI; i += kThreads) {
-          const int pp = i % PI, e = i / PI;
-          const float4 u = NI[(e & 15) * PN + pp], v = NI[(16 + (e >> 4)) * PN + pp];
-          *reinterpret_cast<float4*>(lutI + (e * PI + pp) * 16) =
+      };
+      auto compose = [&](uint8_t* lut, const float4* N, int P) {
+        for (int i = threadIdx.x; i < 128 * P; i += kThreads) {
+          const int pp = i % P, e = i / P;
+          const float4 u = N[(e & 15) * P + pp], v = N[(16 + (e >> 4)) * P + pp];
+          *reinterpret_cast<float4*>(lut + (e * P + pp) * 16) =
               make_float4(u.x + v.x, u.y + v.y, u.z + v.z, u.w + v.w);
         }
-      }
-      for (int i = threadIdx.x; i < Lo::ES * Lo::PS; i += kThreads) {
-        const int pp = i % Lo::PS, e = i / Lo::PS;
-        const float4 u = NS[(e & 15) * Lo::PS + pp], v = NS[(16 + (e >> 4)) * Lo::PS + pp];
-        *reinterpret_cast<float4*>(lutS + (e * Lo::PS + pp) * 16) =
-            make_float4(u.x + v.x, u.y + v.y, u.z + v.z, u.w + v.w);
-      }
+      };
+      if constexpr (Lo::MI == 3) build3(lutI, PI, 0, cenI, cI);
+      else compose(lutI, NI, PI);
+      if constexpr (GRP && Lo::MS == 3) build3(lutS, PS, 32, cenS, cS);
+      else if constexpr (PS > 0) compose(lutS, NS, PS);
     }
     __syncthreads();
 
@@ -436,51 +527,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
 
     for (int ts = c0; ts < t1; ts += kChunkStride) {
       // prefetch the next chunk's key bytes
-      uint32_t nkw[IB / 4], nsw[4], nnw;
+      uint32_t nkw[KW], nsw[4], nnw;
       const int tn = ts + kChunkStride;
       if (tn < t1) load_keys(tn, nkw, nsw, nnw);
       const int wcount = min(32, t1 - ts);
       const bool valid = lane < wcount;
 
       uint64_t accI[2] = {0ull, 0ull}, accS[2] = {0ull, 0ull};
-      if constexpr (PROD) {
-#pragma unroll
-        for (int blk = 0; blk < 2; ++blk) {
-          uint32_t R0, R1;
-          rot_block(sw4[2 * blk], sw4[2 * blk + 1], swap, sh, R0, R1);
-          block_lookups<Lo::PS * 16>(accS, R0, R1, lutS, blk, rot16);
-        }
-      }
-      if constexpr (MB != 3) {
-#pragma unroll
-        for (int blk = 0; blk < IB / 8; ++blk) {
-          uint32_t R0, R1;
-          rot_block(kw[2 * blk], kw[2 * blk + 1], swap, sh, R0, R1);
-          block_lookups<PI * 16>(accI, R0, R1, lutI, blk, rot16);
-        }
-      } else {
-        // bytes of two 3-bit codes: the mirror flips both codes (bit 6 set: high code >= 4)
-#pragma unroll
-        for (int blk = 0; blk < IB / 8; ++blk) {
-          uint32_t R0, R1;
-          rot_block(kw[2 * blk], kw[2 * blk + 1], swap, sh, R0, R1);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint32_t v = ((i < 4 ? R0 : R1) >> (8 * (i & 3))) & 0xffu;
-            const int msk = static_cast<int>(v << 25) >> 31;
-            const uint32_t vc = v ^ (static_cast<uint32_t>(msk) & 0x77u);
-            const uint32_t en = (vc & 7u) | ((vc >> 1) & 0x18u);
-            lut_acc(accI, lutI + 128 * blk + en * (PI * 16) + rot16[i], sign_pair(msk));
-          }
-        }
-      }
-      const float n16 = half_lo(nw), r16 = PROD ? half_hi(nw) : 0.f;
+      if constexpr (PROD) segment_lookups<1, 16>(accS, sw4, lutS, swap, sh, rot16);
+      if constexpr (GRP) segment_lookups<Lo::MS, Lo::PS>(accS, kw + Lo::IBI / 4, lutS, swap, sh, rot16);
+      segment_lookups<Lo::MI, PI>(accI, kw, lutI, swap, sh, rot16);
+      const float n16 = half_lo(nw), r16 = TWO ? half_hi(nw) : 0.f;
       float sc[kMaxHeads];
 #pragma unroll
       for (int j = 0; j < kMaxHeads / 2; ++j) {
         const float2 xi = up2(accI[j]), xs = up2(accS[j]);
-        sc[2 * j] = PROD ? fmaf(n16, xi.x, r16 * xs.x) : n16 * xi.x;
-        sc[2 * j + 1] = PROD ? fmaf(n16, xi.y, r16 * xs.y) : n16 * xi.y;
+        sc[2 * j] = TWO ? fmaf(n16, xi.x, r16 * xs.x) : n16 * xi.x;
+        sc[2 * j + 1] = TWO ? fmaf(n16, xi.y, r16 * xs.y) : n16 * xi.y;
       }
       if (a.scores != nullptr && valid) {
 #pragma unroll
@@ -573,7 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         if (tn < t1) load_values(tn);
       }
 #pragma unroll
-      for (int i = 0; i < IB / 4; ++i) kw[i] = nkw[i];
+      for (int i = 0; i < KW; ++i) kw[i] = nkw[i];
 #pragma unroll
       for (int i = 0; i < 4; ++i) sw4[i] = nsw[i];
       nw = nnw;
@@ -745,10 +808,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
   if (threadIdx.x == 0) a.counters[static_cast<int64_t>(b) * a.n_q_heads + a.g_heads[grp][0]] = 0;
 }
 
-template <int MB, int VB, int NH, bool PROD>
+template <int MB, int VB, int NH, int K>
 tq_status run_decode(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
-  constexpr int smem = Lay<MB, VB, PROD>::total;
-  auto kern = k_decode<MB, VB, NH, PROD>;
+  constexpr int smem = Lay<MB, VB, K>::total;
+  auto kern = k_decode<MB, VB, NH, K>;
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
@@ -770,11 +833,11 @@ tq_status run_decode(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ECUDA;
 }
 
-template <int MB, int VB, bool PROD>
+template <int MB, int VB, int K>
 tq_status run_decode_nh(const DecodeArgs& a, dim3 grid, int max_heads, cudaStream_t st) {
-  if (max_heads <= 2) return run_decode<MB, VB, 2, PROD>(a, grid, st);
-  if (max_heads == 3) return run_decode<MB, VB, 3, PROD>(a, grid, st);
-  return run_decode<MB, VB, 4, PROD>(a, grid, st);
+  if (max_heads <= 2) return run_decode<MB, VB, 2, K>(a, grid, st);
+  if (max_heads == 3) return run_decode<MB, VB, 3, K>(a, grid, st);
+  return run_decode<MB, VB, 4, K>(a, grid, st);
 }
 
 int max_splits_for(int capacity) {
@@ -872,31 +935,41 @@ tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* c, const void*
   a.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + ((parts + 255) / 256) * 256);
 
   const dim3 grid(a.n_splits, n_groups, c->batch);
-  const bool prod = q->mode == TQ_MODE_PROD;
-  const int mb = prod ? q->bits - 1 : q->bits;
+  // MB: index bits (prod: bits - 1) or the grouped base bits
+  const int kind = q->mode == TQ_MODE_PROD ? kProd : (q->mode == TQ_MODE_GROUPED ? kGrp : kMse);
+  const int mb = kind == kProd ? q->bits - 1 : q->bits;
   const int vb = c->value_bits;
-  switch ((prod ? 64 : 0) + mb * 8 + vb) {
-    case 64 + 1 * 8 + 0: return run_decode_nh<1, 0, true>(a, grid, max_heads, st);
-    case 64 + 1 * 8 + 2: return run_decode_nh<1, 2, true>(a, grid, max_heads, st);
-    case 64 + 1 * 8 + 4: return run_decode_nh<1, 4, true>(a, grid, max_heads, st);
-    case 64 + 2 * 8 + 0: return run_decode_nh<2, 0, true>(a, grid, max_heads, st);
-    case 64 + 2 * 8 + 2: return run_decode_nh<2, 2, true>(a, grid, max_heads, st);
-    case 64 + 2 * 8 + 4: return run_decode_nh<2, 4, true>(a, grid, max_heads, st);
-    case 64 + 3 * 8 + 0: return run_decode_nh<3, 0, true>(a, grid, max_heads, st);
-    case 64 + 3 * 8 + 2: return run_decode_nh<3, 2, true>(a, grid, max_heads, st);
-    case 64 + 3 * 8 + 4: return run_decode_nh<3, 4, true>(a, grid, max_heads, st);
-    case 1 * 8 + 0: return run_decode_nh<1, 0, false>(a, grid, max_heads, st);
-    case 1 * 8 + 2: return run_decode_nh<1, 2, false>(a, grid, max_heads, st);
-    case 1 * 8 + 4: return run_decode_nh<1, 4, false>(a, grid, max_heads, st);
-    case 2 * 8 + 0: return run_decode_nh<2, 0, false>(a, grid, max_heads, st);
-    case 2 * 8 + 2: return run_decode_nh<2, 2, false>(a, grid, max_heads, st);
-    case 2 * 8 + 4: return run_decode_nh<2, 4, false>(a, grid, max_heads, st);
-    case 3 * 8 + 0: return run_decode_nh<3, 0, false>(a, grid, max_heads, st);
-    case 3 * 8 + 2: return run_decode_nh<3, 2, false>(a, grid, max_heads, st);
-    case 3 * 8 + 4: return run_decode_nh<3, 4, false>(a, grid, max_heads, st);
-    case 4 * 8 + 0: return run_decode_nh<4, 0, false>(a, grid, max_heads, st);
-    case 4 * 8 + 2: return run_decode_nh<4, 2, false>(a, grid, max_heads, st);
-    case 4 * 8 + 4: return run_decode_nh<4, 4, false>(a, grid, max_heads, st);
+  switch (kind * 64 + mb * 8 + vb) {
+    case kProd * 64 + 1 * 8 + 0: return run_decode_nh<1, 0, kProd>(a, grid, max_heads, st);
+    case kProd * 64 + 1 * 8 + 2: return run_decode_nh<1, 2, kProd>(a, grid, max_heads, st);
+    case kProd * 64 + 1 * 8 + 4: return run_decode_nh<1, 4, kProd>(a, grid, max_heads, st);
+    case kProd * 64 + 2 * 8 + 0: return run_decode_nh<2, 0, kProd>(a, grid, max_heads, st);
+    case kProd * 64 + 2 * 8 + 2: return run_decode_nh<2, 2, kProd>(a, grid, max_heads, st);
+    case kProd * 64 + 2 * 8 + 4: return run_decode_nh<2, 4, kProd>(a, grid, max_heads, st);
+    case kProd * 64 + 3 * 8 + 0: return run_decode_nh<3, 0, kProd>(a, grid, max_heads, st);
+    case kProd * 64 + 3 * 8 + 2: return run_decode_nh<3, 2, kProd>(a, grid, max_heads, st);
+    case kProd * 64 + 3 * 8 + 4: return run_decode_nh<3, 4, kProd>(a, grid, max_heads, st);
+    case kMse * 64 + 1 * 8 + 0: return run_decode_nh<1, 0, kMse>(a, grid, max_heads, st);
+    case kMse * 64 + 1 * 8 + 2: return run_decode_nh<1, 2, kMse>(a, grid, max_heads, st);
+    case kMse * 64 + 1 * 8 + 4: return run_decode_nh<1, 4, kMse>(a, grid, max_heads, st);
+    case kMse * 64 + 2 * 8 + 0: return run_decode_nh<2, 0, kMse>(a, grid, max_heads, st);
+    case kMse * 64 + 2 * 8 + 2: return run_decode_nh<2, 2, kMse>(a, grid, max_heads, st);
+    case kMse * 64 + 2 * 8 + 4: return run_decode_nh<2, 4, kMse>(a, grid, max_heads, st);
+    case kMse * 64 + 3 * 8 + 0: return run_decode_nh<3, 0, kMse>(a, grid, max_heads, st);
+    case kMse * 64 + 3 * 8 + 2: return run_decode_nh<3, 2, kMse>(a, grid, max_heads, st);
+    case kMse * 64 + 3 * 8 + 4: return run_decode_nh<3, 4, kMse>(a, grid, max_heads, st);
+    case kMse * 64 + 4 * 8 + 0: return run_decode_nh<4, 0, kMse>(a, grid, max_heads, st);
+    case kMse * 64 + 4 * 8 + 2: return run_decode_nh<4, 2, kMse>(a, grid, max_heads, st);
+    case kMse * 64 + 4 * 8 + 4: return run_decode_nh<4, 4, kMse>(a, grid, max_heads, st);
+    case kGrp * 64 + 1 * 8 + 0: return run_decode_nh<1, 0, kGrp>(a, grid, max_heads, st);
+    case kGrp * 64 + 1 * 8 + 2: return run_decode_nh<1, 2, kGrp>(a, grid, max_heads, st);
+    case kGrp * 64 + 1 * 8 + 4: return run_decode_nh<1, 4, kGrp>(a, grid, max_heads, st);
+    case kGrp * 64 + 2 * 8 + 0: return run_decode_nh<2, 0, kGrp>(a, grid, max_heads, st);
+    case kGrp * 64 + 2 * 8 + 2: return run_decode_nh<2, 2, kGrp>(a, grid, max_heads, st);
+    case kGrp * 64 + 2 * 8 + 4: return run_decode_nh<2, 4, kGrp>(a, grid, max_heads, st);
+    case kGrp * 64 + 3 * 8 + 0: return run_decode_nh<3, 0, kGrp>(a, grid, max_heads, st);
+    case kGrp * 64 + 3 * 8 + 2: return run_decode_nh<3, 2, kGrp>(a, grid, max_heads, st);
+    case kGrp * 64 + 3 * 8 + 4: return run_decode_nh<3, 4, kGrp>(a, grid, max_heads, st);
     default: return TQ_EUNSUPPORTED;
   }
 }

@@ -279,7 +279,6 @@ static tq_status check_decode_args(const tq_quantizer* q, const tq_kv_cache* c, 
                                    int q_dtype, int n_q_heads, const int32_t* head_map,
                                    void* out, int out_dtype, float* scores, int64_t scores_ld) {
   if (!q) return TQ_EINVAL;
-  if (q->mode == TQ_MODE_GROUPED) return TQ_EUNSUPPORTED;  // prod and mse caches
   tq_status st = check_cache(q, c);
   if (st != TQ_OK) return st;
   if (n_q_heads <= 0 || n_q_heads > 512) return TQ_EINVAL;
@@ -308,7 +307,6 @@ tq_status tq_decode_attention(const tq_quantizer* q, const tq_kv_cache* c, const
                               void* out, int out_dtype, float* scores, int64_t scores_ld,
                               void* workspace, size_t workspace_bytes, void* stream) {
   if (!q) return TQ_EINVAL;
-  if (q->mode == TQ_MODE_GROUPED) return TQ_EUNSUPPORTED;  // prod and mse caches
   tq_status st = check_cache(q, c);
   if (st != TQ_OK) return st;
   if (n_q_heads <= 0 || n_q_heads > 512) return TQ_EINVAL;

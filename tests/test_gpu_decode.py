@@ -84,6 +84,47 @@ def test_decode_mse_scores(bits):
                      O.fp16_from_bits(oc["k_norms"][0, 0, :777, 0]))
 
 
+def grouped_case(seed, B, Hq, Hkv, lengths, cap, bits, vbits):
+    """Keys with 32 fixed high-variance channels (4x std), as in the key-quantize workload."""
+    g = W.rng(seed)
+    N = max(lengths)
+    ch = W.outlier_channels(seed)
+    K = W.round_bf16(W.outlier_rows(g, B * Hkv * N, ch).reshape(B, Hkv, N, 128))
+    V = W.round_bf16(W.gaussian(g, (B, Hkv, N, 128)))
+    Q = W.round_bf16(W.gaussian(g, (B, Hq, 128)))
+    qo = O.build_quantizer(128, bits, "grouped", seed, ch)
+    qg = tq.tq_build_codebook(128, bits, "grouped", seed, ch)
+    oc = oracle_cache(qo, K, V if vbits else None, vbits, lengths)
+    cache = tq.KVCache(qg, B, Hkv, cap, value_bits=vbits, device="cuda:0")
+    upload_cache(cache, oc)
+    return qo, qg, oc, cache, Q
+
+
+@pytest.mark.parametrize("bits,vbits", [(1, 2), (2, 2), (2, 4), (3, 4), (3, 2)])
+def test_decode_grouped_keys(bits, vbits):
+    """grouped caches: s = n_o <Pi_o q_o, c_o[idx_o]> + n_n <Pi_n q_n, c_n[idx_n]> (outlier
+    group at b + 1 bits, normal group at b bits; 20 / 40 / 64 index bytes per key)."""
+    require_cuda()
+    qo, qg, oc, cache, Q = grouped_case(80 + bits, 2, 7, 2, [1100, 613], 1152, bits, vbits)
+    hm = [0, 0, 0, 0, 1, 1, 1]
+    out, _, _ = run_decode(qg, cache, Q, torch.bfloat16, torch.float32, head_map=hm)
+    ref, _ = O.decode_attention(qo, oc, Q.astype(np.float64), head_map=hm, value_bits=vbits)
+    err = check_attention(out, ref, False)
+    print("grouped", bits, vbits, err)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3])
+def test_decode_grouped_scores(bits):
+    require_cuda()
+    qo, qg, oc, cache, Q = grouped_case(90 + bits, 1, 6, 1, [745], 752, bits, 0)
+    _, sc, _ = run_decode(qg, cache, Q, torch.float32, torch.float32, scores_ld=752)
+    _, ref = O.decode_attention(qo, oc, Q.astype(np.float64), value_bits=0, want_scores=True)
+    nrm = O.fp16_from_bits(oc["k_norms"][0, 0, :745])
+    for h in range(6):
+        check_scores(sc[0, h, :745], ref[0][h], np.linalg.norm(Q[0, h]),
+                     np.sqrt(nrm[:, 0] ** 2 + nrm[:, 1] ** 2))
+
+
 def test_decode_head_map_scale_and_scores():
     require_cuda()
     qo, qg, oc, cache, Q = small_case(7, 1, 5, 3, [600], 608, 3, 2)
