@@ -381,7 +381,7 @@ def bench_quantize(tq, torch, dev, world, peak, peak_kind, rows=1 << 22, reps=5,
     out_bytes = lay["idx_bytes"] + lay["sign_bytes"] + 2 * lay["n_norms"]
     gbs = n * (256 + out_bytes) / (ms / 1e3) / 1e9
     kernel = {"prod": f"k_keys_tc<prod,{bits - 1}>", "mse": f"k_keys_tc<mse,{bits}>",
-              "grouped": f"k_keys_grouped<{bits}>"}[mode]
+              "grouped": f"k_keys_grp_tc<{bits}>"}[mode]
     del xs, planes
     torch.cuda.empty_cache()
     return {"rows_per_s": n / (ms / 1e3), "ms_per_pass": ms, "rows_per_pass": n,

@@ -411,6 +411,285 @@ __global__ void __launch_bounds__(128, 2)
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// Grouped keys (tqlite grouped.py; TurboQuant overview, "three quantization modes" table):
+// the 32 outlier channels form a group quantized at b + 1 bits and the other 96 a group at
+// b bits. Each group has its own norm and is rotated by 32-point Hadamard blocks after its
+// own signs; in chain order (outlier channels ascending, then normal channels ascending)
+// block k holds chain positions 32k .. 32k + 31, and u_j > t_k / sqrt(d_g) is decided as
+// y_j > t_k ||x_g|| sqrt(32 / d_g) on the unnormalised block transform y.
+//
+// Same tiling as k_keys_tc (128-row TMA tiles, one thread per row, the transformed row parked
+// in TMEM for a rolled decision loop), with a gather in front: once a tile has landed, each
+// warp copies its 32 rows into chain order in a padded shared-memory buffer (lane l moves
+// the natural channels 4l .. 4l + 3 of a row), which also releases the TMA buffer. The four
+// transforms run on fp32 pairs (y_p, y_{p+64}): blocks 0 and 2 share pair indices 0..31,
+// blocks 1 and 3 pair indices 32..63, so every butterfly is one packed add or subtract.
+// ---------------------------------------------------------------------------------------
+constexpr int kGStride = 272;                    // bytes per chain-ordered row (256 + 16)
+constexpr int kGPermOff = 2 * kXBuf;
+constexpr int kGMaskOff = kGPermOff + kTile * kGStride;
+constexpr int kGPosOff = kGMaskOff + 256;        // chain position of each channel (uint16)
+constexpr int kGCodeOff = kGPosOff + 256;        // packed halfwords [32][kTile] (uint16)
+constexpr int kGSmemBytes = kGCodeOff + 32 * kTile * 2;
+
+// Codes of 16 values (pairs i, i + 8 of yv) against NT ascending thresholds, packed
+// LSB-first at width W into W halfwords sCode[(hw0 + j) kTile + tid], j < W. Exact 0/1
+// compares are summed with power-of-two weights as exact fp32 integers below 2^16.
+template <int W, int NT>
+__device__ __forceinline__ void decide16(const uint32_t (&yv)[16], const float (&T)[NT],
+                                         uint16_t* sCode, int hw0, int tid) {
+  constexpr int NA = W == 4 ? 2 : 1;
+  uint64_t acc[NA];
+#pragma unroll
+  for (int j = 0; j < NA; ++j) acc[j] = pk2(0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int slot = W == 4 ? 4 * (i & 3) : W * i;
+    const float wx = static_cast<float>(1u << slot);
+    const float wy = W == 1 ? static_cast<float>(1u << (i + 8)) : wx;
+    const uint64_t kw = pk2(wx, wy);
+    const float y0 = __uint_as_float(yv[i]), y1 = __uint_as_float(yv[i + 8]);
+    uint64_t& A = acc[W == 4 ? i / 4 : 0];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) A = fma2(pk2(gt_one(y0, T[t]), gt_one(y1, T[t])), kw, A);
+  }
+  auto bits16 = [](float f) {  // an exact integer below 2^16 lands in the low mantissa bits
+    return static_cast<uint16_t>(__float_as_uint(f + 8388608.f) & 0xffffu);
+  };
+  if constexpr (W == 1) {
+    const float2 v = up2(acc[0]);
+    sCode[hw0 * kTile + tid] = bits16(v.x + v.y);
+  } else if constexpr (W == 2) {
+    const float2 v = up2(acc[0]);
+    sCode[hw0 * kTile + tid] = bits16(v.x);
+    sCode[(hw0 + 1) * kTile + tid] = bits16(v.y);
+  } else {
+    const float2 v0 = up2(acc[0]), v1 = up2(acc[1]);
+    sCode[hw0 * kTile + tid] = bits16(v0.x);
+    sCode[(hw0 + 1) * kTile + tid] = bits16(v1.x);
+    sCode[(hw0 + 2) * kTile + tid] = bits16(v0.y);
+    sCode[(hw0 + 3) * kTile + tid] = bits16(v1.y);
+  }
+}
+
+template <int B>
+__global__ void __launch_bounds__(128, 2)
+    k_keys_grp_tc(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ TcKeyArgs a) {
+  constexpr int NTO = (1 << (B + 1)) - 1, NTN = (1 << B) - 1;
+  constexpr int WO = storage_width_c(B + 1), WN = storage_width_c(B);
+  constexpr int HWO = 2 * WO;           // halfwords of the outlier group (32 codes)
+  constexpr int NHW = HWO + 6 * WN;     // halfwords per row
+  constexpr int IB = 2 * NHW;           // index bytes per row: 20, 40, 64
+
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* sX = smem;
+  uint8_t* sP = smem + kGPermOff;
+  const uint32_t* sMask = reinterpret_cast<const uint32_t*>(smem + kGMaskOff);
+  uint16_t* sPos = reinterpret_cast<uint16_t*>(smem + kGPosOff);
+  uint16_t* sCode = reinterpret_cast<uint16_t*>(smem + kGCodeOff);
+  __shared__ __align__(8) uint64_t bar_x[2];
+  __shared__ __align__(8) uint64_t bar_b;
+  __shared__ __align__(8) uint64_t bar_free[2];  // every thread has gathered from buffer b
+  __shared__ uint32_t tslot;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const DevTables* __restrict__ tab = a.tab;
+  const int64_t grid = gridDim.x;
+  const int64_t n_local = (a.n_tiles - blockIdx.x + grid - 1) / grid;  // grid <= n_tiles
+
+  if (warp == 0) {
+    tmem_alloc(&tslot, 128u);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&bar_x[0], 1);
+    mbar_init(&bar_x[1], 1);
+    mbar_init(&bar_b, 1);
+    mbar_init(&bar_free[0], kTile);
+    mbar_init(&bar_free[1], kTile);
+    fence_mbar_init();
+  }
+  sPos[tab->chan[tid]] = static_cast<uint16_t>(tid);  // chan is a permutation of 0..127
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tlane = tslot + (static_cast<uint32_t>(warp * 32) << 16);
+
+  if (tid == 0) {
+    mbar_expect_tx(&bar_b, 256);
+    bulk_g2s(smem + kGMaskOff, tab->pair_mask, 256, &bar_b);
+    for (int k = 0; k < 2 && k < n_local; ++k) {
+      const int row0 = static_cast<int>((blockIdx.x + k * grid) * kTile);
+      mbar_expect_tx(&bar_x[k], kXBuf);
+      tma_load_2d(sX + k * kXBuf, &tmap, 0, row0, &bar_x[k]);
+      tma_load_2d(sX + k * kXBuf + kXBuf / 2, &tmap, 64, row0, &bar_x[k]);
+    }
+  }
+
+  // byte offsets, in a chain-ordered row, of this lane's natural channels 4 lane .. 4 lane + 3
+  uint32_t dpos[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) dpos[i] = 2u * sPos[4 * lane + i];
+  // where those channels sit in a staged (swizzled) row: 64-column half lane / 16, 16-byte
+  // chunk (lane mod 16) / 2, 8-byte half lane mod 2
+  const uint32_t src_off = (lane >> 4) * (kXBuf / 2) + (lane & 1) * 8;
+  const uint32_t src_c = static_cast<uint32_t>((lane & 15) >> 1);
+  float thrO[NTO], thrN[NTN];
+#pragma unroll
+  for (int t = 0; t < NTO; ++t) thrO[t] = tab->thr[0][t];
+#pragma unroll
+  for (int t = 0; t < NTN; ++t) thrN[t] = tab->thr[1][t];
+
+  bool ok = mbar_wait_ns(&bar_b, 0, kWaitNs);
+  for (int64_t k = 0; k < n_local; ++k) {
+    const int b = static_cast<int>(k & 1);
+    const int64_t tile = blockIdx.x + k * grid;
+    const int64_t row = tile * kTile + tid;
+    const bool valid = row < a.n_rows;
+    if (ok) ok = mbar_wait_ns(&bar_x[b], static_cast<uint32_t>((k >> 1) & 1), kWaitNs);
+
+    // ---- gather this warp's 32 rows into chain order
+    __syncwarp();  // the warp's lanes are done reading their rows of the previous tile
+    {
+      const uint8_t* src = sX + b * kXBuf + src_off;
+#pragma unroll 4
+      for (int j = 0; j < 32; ++j) {
+        const int r = warp * 32 + j;
+        const uint2 v = *reinterpret_cast<const uint2*>(src + r * 128 + ((src_c ^ static_cast<uint32_t>(r & 7)) << 4));
+        uint8_t* dst = sP + r * kGStride;
+        *reinterpret_cast<uint16_t*>(dst + dpos[0]) = static_cast<uint16_t>(v.x);
+        *reinterpret_cast<uint16_t*>(dst + dpos[1]) = static_cast<uint16_t>(v.x >> 16);
+        *reinterpret_cast<uint16_t*>(dst + dpos[2]) = static_cast<uint16_t>(v.y);
+        *reinterpret_cast<uint16_t*>(dst + dpos[3]) = static_cast<uint16_t>(v.y >> 16);
+      }
+    }
+    mbar_arrive(&bar_free[b]);
+    __syncwarp();
+
+    // ---- own row: signs, the two norms, four 32-point transforms on (y_p, y_{p+64}) pairs
+    uint64_t P[64];
+    uint64_t na[4], nb[4];  // sums of squares: na pairs p < 32 (.x outliers), nb p >= 32
+#pragma unroll
+    for (int i = 0; i < 4; ++i) na[i] = nb[i] = pk2(0.f, 0.f);
+    {
+      const uint8_t* x0 = sP + tid * kGStride;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 u0 = *reinterpret_cast<const uint4*>(x0 + 16 * c);
+        const uint4 u1 = *reinterpret_cast<const uint4*>(x0 + 128 + 16 * c);
+        const uint4 m0 = *reinterpret_cast<const uint4*>(sMask + 4 * c);
+        const uint4 m1 = *reinterpret_cast<const uint4*>(sMask + 32 + 4 * c);
+        const uint32_t wl[4] = {u0.x ^ m0.x, u0.y ^ m0.y, u0.z ^ m0.z, u0.w ^ m0.w};
+        const uint32_t wh[4] = {u1.x ^ m1.x, u1.y ^ m1.y, u1.z ^ m1.z, u1.w ^ m1.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int p = 8 * c + 2 * i;
+          P[p] = pk2(__uint_as_float(wl[i] << 16), __uint_as_float(wh[i] << 16));
+          P[p + 1] = pk2(__uint_as_float(wl[i] & 0xffff0000u), __uint_as_float(wh[i] & 0xffff0000u));
+          if (c < 4) {
+            na[i] = fma2(P[p], P[p], na[i]);
+            na[i] = fma2(P[p + 1], P[p + 1], na[i]);
+          } else {
+            nb[i] = fma2(P[p], P[p], nb[i]);
+            nb[i] = fma2(P[p + 1], P[p + 1], nb[i]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+      for (int p = 0; p < 64; ++p) {
+        if ((p & h) == 0) {
+          const uint64_t u = P[p], v = P[p + h];
+          P[p] = add2(u, v);
+          P[p + h] = sub2(u, v);
+        }
+      }
+    }
+    const float2 sa = up2(add2(add2(na[0], na[1]), add2(na[2], na[3])));
+    const float2 sb = up2(add2(add2(nb[0], nb[1]), add2(nb[2], nb[3])));
+    const float n_o = sqrtf(sa.x), n_n = sqrtf(sa.y + (sb.x + sb.y));
+    const __half no16 = __float2half_rn(n_o), nn16 = __float2half_rn(n_n);
+
+    // ---- park the transformed row: chain position c -> TMEM column c
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      uint32_t r[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 v = up2(P[16 * (q & 3) + i]);
+        r[i] = __float_as_uint(q < 4 ? v.x : v.y);
+      }
+      tmem_st16(tlane + 16 * q, r);
+    }
+    tmem_st_wait();
+
+    // ---- decisions: the outlier group (2 units of 16), then the normal group (6 units)
+    float TO[NTO], TN[NTN];
+    const float ns = n_n * 0.57735026918962576f;  // sqrt(32 / 96)
+#pragma unroll
+    for (int t = 0; t < NTO; ++t) TO[t] = n_o > 0.f ? thrO[t] * n_o : thrO[t];
+#pragma unroll
+    for (int t = 0; t < NTN; ++t) TN[t] = n_n > 0.f ? thrN[t] * ns : thrN[t];
+#pragma unroll 1
+    for (int u = 0; u < 2; ++u) {
+      uint32_t yv[16];
+      tmem_ld16_sync(tlane + 16 * u, yv);
+      decide16<WO, NTO>(yv, TO, sCode, u * WO, tid);
+    }
+#pragma unroll 1
+    for (int u = 0; u < 6; ++u) {
+      uint32_t yv[16];
+      tmem_ld16_sync(tlane + 32 + 16 * u, yv);
+      decide16<WN, NTN>(yv, TN, sCode, HWO + u * WN, tid);
+    }
+
+    if (valid) {
+      const int64_t orow = out_row_tc(a.map, a.row_base + row);
+      uint32_t w[NHW / 2];
+#pragma unroll
+      for (int i = 0; i < NHW / 2; ++i)
+        w[i] = static_cast<uint32_t>(sCode[2 * i * kTile + tid]) |
+               (static_cast<uint32_t>(sCode[(2 * i + 1) * kTile + tid]) << 16);
+      uint8_t* dst = a.idx + orow * IB;
+      if constexpr (IB % 16 == 0) {
+#pragma unroll
+        for (int i = 0; i < IB / 16; ++i)
+          reinterpret_cast<uint4*>(dst)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+      } else if constexpr (IB % 8 == 0) {
+#pragma unroll
+        for (int i = 0; i < IB / 8; ++i) reinterpret_cast<uint2*>(dst)[i] = make_uint2(w[2 * i], w[2 * i + 1]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < IB / 4; ++i) reinterpret_cast<uint32_t*>(dst)[i] = w[i];
+      }
+      a.nrm[orow * 2] = half_bits(no16);
+      a.nrm[orow * 2 + 1] = half_bits(nn16);
+    }
+
+    // ---- refill staging buffer b two tiles ahead once every thread has gathered from it
+    if (tid == 0 && ok && k + 2 < n_local) {
+      ok = mbar_wait_ns(&bar_free[b], static_cast<uint32_t>((k >> 1) & 1), kWaitNs);
+      if (ok) {
+        const int row0 = static_cast<int>((tile + 2 * grid) * kTile);
+        mbar_expect_tx(&bar_x[b], kXBuf);
+        tma_load_2d(sX + b * kXBuf, &tmap, 0, row0, &bar_x[b]);
+        tma_load_2d(sX + b * kXBuf + kXBuf / 2, &tmap, 64, row0, &bar_x[b]);
+      }
+    }
+  }
+
+  if (!ok) atomicOr(a.err, 1);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tslot, 128u);
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -442,13 +721,30 @@ tq_status run_tc(const CUtensorMap& tmap, const TcKeyArgs& a, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ECUDA;
 }
 
+template <int B>
+tq_status run_grp_tc(const CUtensorMap& tmap, const TcKeyArgs& a, cudaStream_t st) {
+  auto kern = k_keys_grp_tc<B>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmemBytes) !=
+        cudaSuccess)
+      return TQ_ECUDA;
+    attr_set = true;
+  }
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int64_t cap = 2ll * sm_count(dev);
+  const int grid = static_cast<int>(a.n_tiles < cap ? a.n_tiles : cap);
+  kern<<<grid, 128, kGSmemBytes, st>>>(tmap, a);
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ECUDA;
+}
+
 }  // namespace
 
 __device__ int g_tq_device_error = 0;
 
 bool keys_tc_ok(const tq_quantizer* q, int dtype) {
-  return (q->mode == TQ_MODE_PROD || q->mode == TQ_MODE_MSE) && dtype == TQ_BF16 &&
-         encode_fn() != nullptr;
+  return dtype == TQ_BF16 && encode_fn() != nullptr;
 }
 
 tq_status launch_keys_tc(const tq_quantizer* q, const void* x, int64_t n_rows, int64_t ld,
@@ -474,7 +770,10 @@ tq_status launch_keys_tc(const tq_quantizer* q, const void* x, int64_t n_rows, i
       return TQ_ECUDA;
     TcKeyArgs a{nr, r0, (nr + kTile - 1) / kTile, q->dev, out.idx, out.signs, out.norms, map, err};
     tq_status s;
-    switch ((q->mode == TQ_MODE_PROD ? 8 : 0) + q->bits) {
+    switch ((q->mode == TQ_MODE_PROD ? 8 : (q->mode == TQ_MODE_GROUPED ? 16 : 0)) + q->bits) {
+      case 16 + 1: s = run_grp_tc<1>(tmap, a, st); break;
+      case 16 + 2: s = run_grp_tc<2>(tmap, a, st); break;
+      case 16 + 3: s = run_grp_tc<3>(tmap, a, st); break;
       case 8 + 2: s = run_tc<true, 1>(tmap, a, st); break;
       case 8 + 3: s = run_tc<true, 2>(tmap, a, st); break;
       case 8 + 4: s = run_tc<true, 3>(tmap, a, st); break;
