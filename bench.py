@@ -68,6 +68,10 @@ def parse():
                     help="decode workload of the timed step (the headline line is decode-s)")
     ap.add_argument("--quantize-sweep", action="store_true",
                     help="with --only quantize: every mode and width of the key-quantize sweep")
+    ap.add_argument("--quantize-mode", default="prod3",
+                    choices=["mse1", "mse2", "mse3", "mse4", "prod2", "prod3", "prod4",
+                             "grouped1", "grouped2", "grouped3"],
+                    help="with --only quantize: the mode and width of the single timed pass")
     return ap.parse_args()
 
 
@@ -209,7 +213,9 @@ def run_tq(args):
             if rank == 0:
                 print(json.dumps({"key_quantize_sweep": out}))
             return
-        r = bench_quantize(tq, torch, dev, world, peak, peak_kind, rows=args.quantize_rows)
+        qm = args.quantize_mode
+        r = bench_quantize(tq, torch, dev, world, peak, peak_kind, rows=args.quantize_rows,
+                           mode=qm[:-1], bits=int(qm[-1]))
         if rank == 0:
             print(json.dumps({"key_quantize": r}))
         return

@@ -283,6 +283,20 @@ __global__ void __launch_bounds__(128, 2)
     }
     const uint64_t ncs02 = pk2(ncs[0], ncs[0]);
     const uint64_t scl2 = pk2(scl, scl);
+    // Symmetric codebooks (C_{L-1-k} = -C_k, t_{L-2-k} = -t_k, middle threshold 0), used for
+    // L >= 8: with s = [y > 0], sigma = 2 s - 1 and m = #{t < H : |y| > T+_t} over the
+    // H = L/2 - 1 positive thresholds, code = (L - 1)/2 + sigma (m + 1/2) and the centroid is
+    // sigma C+_m. (|y| on a positive threshold, a tie, may take the neighbouring code.)
+    constexpr bool SYM = NL >= 8;
+    constexpr int H = NL / 2 - 1;
+    float TP[SYM ? H : 1];
+    uint64_t dcsP2[SYM ? H : 1];
+#pragma unroll
+    for (int t = 0; t < H; ++t) {
+      TP[t] = T[NL / 2 + t];
+      dcsP2[t] = pk2(ncs[NL / 2 + t + 1] - ncs[NL / 2 + t], ncs[NL / 2 + t + 1] - ncs[NL / 2 + t]);
+    }
+    const uint64_t ncsP02 = pk2(ncs[NL / 2], ncs[NL / 2]);
     const uint64_t kSplit2 = pk2(8192.f, 8192.f);  // c = 8192 r + r
 
     uint64_t racc[4];
@@ -292,7 +306,9 @@ __global__ void __launch_bounds__(128, 2)
     for (int g = 0; g < NG; ++g) {
       // index words of elements [GP g, GP g + GP) (.x) and +64 (.y), accumulated in fp32 as
       // exact integers: codes of pairs [0, GP/2) in wa, [GP/2, GP) in wb (each < 2^16)
-      uint64_t wa = pk2(0.f, 0.f), wb = pk2(0.f, 0.f);
+      // symmetric path: each word starts at sum_j kw_j (L - 1)/2 over its pairs
+      constexpr float kW0 = SYM ? 0.5f * (NL - 1) * (W == 4 ? 4369.f : W == 2 ? 21845.f : 65535.f) : 0.f;
+      uint64_t wa = pk2(kW0, kW0), wb = pk2(kW0, kW0);
       uint32_t hw[GP], lw[GP];
 #pragma unroll
       for (int q = 0; q < GP / 8; ++q) {
@@ -306,18 +322,36 @@ __global__ void __launch_bounds__(128, 2)
           const float kw = static_cast<float>(1u << (W * (pi % (GP / 2))));
           const uint64_t kw2 = pk2(kw, kw);
           const uint64_t y2 = pk2(__uint_as_float(yv[2 * i]), __uint_as_float(yv[2 * i + 1]));
-          uint64_t c2 = ncs02;
+          uint64_t c2 = SYM ? ncsP02 : ncs02;
+          uint64_t sg2 = 0ull;
+          if constexpr (SYM) {
+            const float y0 = __uint_as_float(yv[2 * i]), y1 = __uint_as_float(yv[2 * i + 1]);
+            const uint64_t s2 = pk2(gt_one(y0, 0.f), gt_one(y1, 0.f));
+            const uint64_t sk2 = fma2(s2, pk2(2.f * kw, 2.f * kw), pk2(-kw, -kw));  // sigma kw
+            uint64_t w = fma2(sk2, pk2(0.5f, 0.5f), pi < GP / 2 ? wa : wb);
+            const float a0 = fabsf(y0), a1 = fabsf(y1);
 #pragma unroll
-          for (int t = 0; t < NL - 1; ++t) {
-            const float2 th = up2(T2[t]);
-            const uint64_t ind = pk2(gt_one(__uint_as_float(yv[2 * i]), th.x),
-                                     gt_one(__uint_as_float(yv[2 * i + 1]), th.y));
-            if constexpr (PROD) c2 = fma2(ind, dcs2[t], c2);
-            if (pi < GP / 2) wa = fma2(ind, kw2, wa);
-            else wb = fma2(ind, kw2, wb);
+            for (int t = 0; t < H; ++t) {
+              const uint64_t ind = pk2(gt_one(a0, TP[t]), gt_one(a1, TP[t]));
+              if constexpr (PROD) c2 = fma2(ind, dcsP2[t], c2);
+              w = fma2(ind, sk2, w);
+            }
+            if (pi < GP / 2) wa = w;
+            else wb = w;
+            if constexpr (PROD) sg2 = fma2(s2, pk2(2.f, 2.f), pk2(-1.f, -1.f));
+          } else {
+#pragma unroll
+            for (int t = 0; t < NL - 1; ++t) {
+              const float2 th = up2(T2[t]);
+              const uint64_t ind = pk2(gt_one(__uint_as_float(yv[2 * i]), th.x),
+                                       gt_one(__uint_as_float(yv[2 * i + 1]), th.y));
+              if constexpr (PROD) c2 = fma2(ind, dcs2[t], c2);
+              if (pi < GP / 2) wa = fma2(ind, kw2, wa);
+              else wb = fma2(ind, kw2, wb);
+            }
           }
           if constexpr (!PROD) continue;
-          const uint64_t r = fma2(y2, scl2, c2);
+          const uint64_t r = SYM ? fma2(sg2, c2, mul2(y2, scl2)) : fma2(y2, scl2, c2);
           racc[pi & 3] = fma2(r, r, racc[pi & 3]);
           // Veltkamp split: hi keeps the top 11 significant bits (exact in fp16 for |r| < 2^15),
           // lo = r - hi exactly (13 bits, rounded to fp16's 11). c = RN(8193 r) comes from one
@@ -440,9 +474,13 @@ template <int W, int NT>
 __device__ __forceinline__ void decide16(const uint32_t (&yv)[16], const float (&T)[NT],
                                          uint16_t* sCode, int hw0, int tid) {
   constexpr int NA = W == 4 ? 2 : 1;
+  // L = NT + 1 >= 8 (4-bit fields): symmetric codebook, code = (L - 1)/2 + sigma (m + 1/2)
+  // with m counted on |y| against the H positive thresholds (as in k_keys_tc)
+  constexpr bool SYM = NT >= 7;
+  constexpr int H = (NT + 1) / 2 - 1;
   uint64_t acc[NA];
 #pragma unroll
-  for (int j = 0; j < NA; ++j) acc[j] = pk2(0.f, 0.f);
+  for (int j = 0; j < NA; ++j) acc[j] = SYM ? pk2(0.5f * NT * 4369.f, 0.5f * NT * 4369.f) : pk2(0.f, 0.f);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int slot = W == 4 ? 4 * (i & 3) : W * i;
@@ -451,8 +489,17 @@ __device__ __forceinline__ void decide16(const uint32_t (&yv)[16], const float (
     const uint64_t kw = pk2(wx, wy);
     const float y0 = __uint_as_float(yv[i]), y1 = __uint_as_float(yv[i + 8]);
     uint64_t& A = acc[W == 4 ? i / 4 : 0];
+    if constexpr (SYM) {
+      const uint64_t s2 = pk2(gt_one(y0, 0.f), gt_one(y1, 0.f));
+      const uint64_t sk2 = fma2(s2, pk2(2.f * wx, 2.f * wx), pk2(-wx, -wx));  // sigma kw
+      A = fma2(sk2, pk2(0.5f, 0.5f), A);
+      const float a0 = fabsf(y0), a1 = fabsf(y1);
 #pragma unroll
-    for (int t = 0; t < NT; ++t) A = fma2(pk2(gt_one(y0, T[t]), gt_one(y1, T[t])), kw, A);
+      for (int t = 0; t < H; ++t) A = fma2(pk2(gt_one(a0, T[H + 1 + t]), gt_one(a1, T[H + 1 + t])), sk2, A);
+    } else {
+#pragma unroll
+      for (int t = 0; t < NT; ++t) A = fma2(pk2(gt_one(y0, T[t]), gt_one(y1, T[t])), kw, A);
+    }
   }
   auto bits16 = [](float f) {  // an exact integer below 2^16 lands in the low mantissa bits
     return static_cast<uint16_t>(__float_as_uint(f + 8388608.f) & 0xffffu);
