@@ -230,6 +230,32 @@ tq_status tq_decode_attention_noalloc(const tq_quantizer* q, const tq_kv_cache* 
                                       void* out_dev, int out_dtype,
                                       float* scores_dev, int64_t scores_ld, void* stream);
 
+/* ---- context-parallel decode (a cache's context split into slices, e.g. one per GPU) ----
+ * Softmax attention over the union of the slices equals the LSE merge of per-slice partial
+ * results (the merge the fused decode kernel already runs between its own context splits):
+ *   step 1, per slice:  tq_decode_attention_partial -> (m, l, o) per (sequence, query head)
+ *   exchange:           gather every slice's records (an all-gather across GPUs)
+ *   step 2:             tq_merge_partials -> out = sum 2^(m_r - M) o_r / sum 2^(m_r - M) l_r
+ * A record is TQ_PART_FLOATS fp32 values: m (the largest logit, base 2: sm_scale log2(e) s),
+ * l = sum_i 2^(x_i - m), two zeros, and the unnormalised o = sum_i 2^(x_i - m) v_hat_i [d].
+ * An empty slice (len[b] = 0) gives m = -inf, l = 0, o = 0. */
+#define TQ_PART_FLOATS 132
+
+/* Step 1: as tq_decode_attention (same arguments, checks and workspace) on a cache with
+ * values, writing the records to part_dev (fp32 batch x n_q_heads x TQ_PART_FLOATS,
+ * 16-byte aligned) instead of normalised outputs. */
+tq_status tq_decode_attention_partial(const tq_quantizer* q, const tq_kv_cache* cache,
+                                      const void* q_dev, int q_dtype, int n_q_heads,
+                                      const int32_t* head_map, float sm_scale, float* part_dev,
+                                      void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/* Step 2: merge n_parts (1 .. 65536) slices' records, parts_dev = fp32 n_parts x batch x
+ * n_q_heads x TQ_PART_FLOATS (16-byte aligned; slices may come in any order), into out_dev
+ * (batch x n_q_heads x d, TQ_F32 or TQ_BF16, 16-byte aligned). All slices must have used the
+ * same sm_scale. */
+tq_status tq_merge_partials(const float* parts_dev, int n_parts, int batch, int n_q_heads,
+                            void* out_dev, int out_dtype, void* stream);
+
 /* Wait for `stream` (cudaStream_t as void*, NULL = legacy default stream) and report whether
  * any library kernel since the previous call gave up one of its bounded device waits (an
  * mbarrier wait on a bulk copy or a tensor-core product, limit 2 s): TQ_ETIMEOUT if so (the

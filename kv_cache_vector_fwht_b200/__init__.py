@@ -29,7 +29,8 @@ D = 128
 
 EXPORTED = ["tq_build_codebook", "tq_free", "tq_key_layout", "tq_host_tables",
             "tq_quantize_keys", "tq_dequantize_keys", "tq_quantize_values", "tq_append", "tq_decode_workspace_bytes",
-            "tq_decode_attention", "tq_decode_attention_noalloc", "tq_sync_status",
+            "tq_decode_attention", "tq_decode_attention_noalloc", "tq_decode_attention_partial",
+            "tq_merge_partials", "tq_sync_status",
             "tq_selftest_bounded_wait", "tq_status_string", "tq_abi_version"]
 
 
@@ -86,6 +87,12 @@ _lib.tq_decode_attention_noalloc.argtypes = [c_void_p, POINTER(KVCacheDesc), c_v
                                              c_int, POINTER(c_int32), c_float, c_void_p, c_int,
                                              c_void_p, c_int64, c_void_p]
 _lib.tq_decode_attention_noalloc.restype = c_int
+_lib.tq_decode_attention_partial.argtypes = [c_void_p, POINTER(KVCacheDesc), c_void_p, c_int,
+                                             c_int, POINTER(c_int32), c_float, c_void_p,
+                                             c_void_p, c_size_t, c_void_p]
+_lib.tq_decode_attention_partial.restype = c_int
+_lib.tq_merge_partials.argtypes = [c_void_p, c_int, c_int, c_int, c_void_p, c_int, c_void_p]
+_lib.tq_merge_partials.restype = c_int
 _lib.tq_status_string.argtypes = [c_int]
 _lib.tq_status_string.restype = ctypes.c_char_p
 _lib.tq_abi_version.argtypes = []
@@ -333,6 +340,33 @@ def tq_decode_attention(q: Quantizer, cache: KVCache, query, out=None, workspace
                                     _dtype_code(out) if out is not None else TQ_F32,
                                     _ptr(scores), sld, _ptr(workspace), wbytes, _stream(stream)),
            "tq_decode_attention")
+
+
+TQ_PART_FLOATS = 132   # floats per partial record: m, l, 0, 0, o[128]
+
+
+def tq_decode_attention_partial(q: Quantizer, cache: KVCache, query, part, workspace,
+                                head_map=None, sm_scale: float = 0.0, stream=None) -> None:
+    """One context slice of a context-parallel decode: part (batch, n_q_heads, TQ_PART_FLOATS)
+    fp32 receives this cache's (m, l, o) records (see tq.h)."""
+    assert query.is_contiguous() and query.dim() == 3
+    assert part.is_contiguous() and part.shape[-1] == TQ_PART_FLOATS
+    hq = query.shape[1]
+    hm = (c_int32 * hq)(*[int(v) for v in head_map]) if head_map is not None else None
+    _check(_lib.tq_decode_attention_partial(q.handle, ctypes.byref(cache.desc), _ptr(query),
+                                            _dtype_code(query), hq, hm, sm_scale, _ptr(part),
+                                            _ptr(workspace), workspace.numel(), _stream(stream)),
+           "tq_decode_attention_partial")
+
+
+def tq_merge_partials(parts, out, stream=None) -> None:
+    """parts: (n_parts, batch, n_q_heads, TQ_PART_FLOATS) fp32, contiguous; out: (batch,
+    n_q_heads, d) fp32/bf16 receives the LSE merge of the slices."""
+    assert parts.is_contiguous() and parts.dim() == 4 and parts.shape[-1] == TQ_PART_FLOATS
+    assert out.is_contiguous() and tuple(out.shape[:2]) == tuple(parts.shape[1:3])
+    _check(_lib.tq_merge_partials(_ptr(parts), parts.shape[0], parts.shape[1], parts.shape[2],
+                                  _ptr(out), _dtype_code(out), _stream(stream)),
+           "tq_merge_partials")
 
 
 def tq_decode_attention_noalloc(q: Quantizer, cache: KVCache, query, out=None, head_map=None,

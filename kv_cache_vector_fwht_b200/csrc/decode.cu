@@ -58,6 +58,7 @@ struct DecodeArgs {
   const void* q;
   void* out;
   float* scores;
+  float* part_out;  // nullable: per (sequence, query head) (m, l, o) records instead of out
   float* part;
   int* counters;
   const DevTables* tab;
@@ -691,7 +692,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
       }
     }
     const int64_t orow = (static_cast<int64_t>(b) * a.n_q_heads + hq) * kD + 4 * lane;
-    if (a.n_splits == 1) {
+    if (a.n_splits == 1 && a.part_out != nullptr) {
+      float* dst = a.part_out + (static_cast<int64_t>(b) * a.n_q_heads + hq) * kPartStride;
+      if (lane == 0) *reinterpret_cast<float4*>(dst) = make_float4(M, Lsum, 0.f, 0.f);
+      *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = make_float4(O[0], O[1], O[2], O[3]);
+    } else if (a.n_splits == 1) {
       const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
       if (a.out_f32) {
         *reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow) =
@@ -730,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     float* sMx = reinterpret_cast<float*>(smem + Lo::wv);   // [head][S] split maxima
     float* sLs = sMx + kMaxHeads * 256;                      // [head][S] split sums
     float* sF = sLs + kMaxHeads * 256;                       // [head][S] weights
-    float* sHd = sF + kMaxHeads * 256;                       // [head]: 1 / total sum
+    float* sHd = sF + kMaxHeads * 256;  // [head] 1 / total sum, then [head] maxima and sums
     float4* sAcc = reinterpret_cast<float4*>(sHd + 16);      // [slice][head][32]
     const float* base = a.part + static_cast<int64_t>(b) * a.n_q_heads * S * kPartStride;
     for (int i = threadIdx.x; i < nh * S; i += kThreads) {
@@ -753,7 +758,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         lsum = fmaf(f, sLs[h * 256 + sp], lsum);
       }
       lsum = warp_sum(lsum);
-      if (lane == 0) sHd[h] = lsum > 0.f ? 1.f / lsum : 0.f;
+      if (lane == 0) {
+        sHd[h] = lsum > 0.f ? 1.f / lsum : 0.f;
+        sHd[kMaxHeads + h] = M;
+        sHd[2 * kMaxHeads + h] = lsum;
+      }
     }
     __syncthreads();
     const int G = kThreads / (32 * nh);  // split slices
@@ -792,7 +801,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
       }
       const float inv = sHd[h];
       const int64_t orow = (static_cast<int64_t>(b) * a.n_q_heads + hq) * kD + 4 * qd;
-      if (a.out_f32) {
+      if (a.part_out != nullptr) {
+        float* dst = a.part_out + (static_cast<int64_t>(b) * a.n_q_heads + hq) * kPartStride;
+        if (qd == 0) *reinterpret_cast<float4*>(dst) = make_float4(sHd[kMaxHeads + h], sHd[2 * kMaxHeads + h], 0.f, 0.f);
+        *reinterpret_cast<float4*>(dst + 4 + 4 * qd) = O;
+      } else if (a.out_f32) {
         *reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow) =
             make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
       } else {
@@ -840,12 +853,60 @@ tq_status run_decode_nh(const DecodeArgs& a, dim3 grid, int max_heads, cudaStrea
   return run_decode<MB, VB, 4, K>(a, grid, st);
 }
 
+// LSE merge of context-split partial records (m, l, o) of n_parts slices: per row (sequence,
+// query head) M = max m_r, out = sum 2^(m_r - M) o_r / sum 2^(m_r - M) l_r (zeros when every
+// slice is empty). One warp per row, lane l owns channels 4l .. 4l + 3.
+__global__ void __launch_bounds__(128) k_merge_partials(const float* __restrict__ parts, int n_parts,
+                                                        int64_t rows, void* out, int out_f32) {
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float M = -INFINITY;
+  for (int r = 0; r < n_parts; ++r) M = fmaxf(M, __ldg(parts + (r * rows + row) * kPartStride));
+  float L = 0.f;
+  float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (M != -INFINITY) {
+    for (int r = 0; r < n_parts; ++r) {
+      const float* rec = parts + (r * rows + row) * kPartStride;
+      const float mr = __ldg(rec);
+      if (mr == -INFINITY) continue;
+      const float f = exp2f(mr - M);
+      L = fmaf(f, __ldg(rec + 1), L);
+      const float4 v = __ldg(reinterpret_cast<const float4*>(rec + 4) + lane);
+      O.x = fmaf(f, v.x, O.x); O.y = fmaf(f, v.y, O.y);
+      O.z = fmaf(f, v.z, O.z); O.w = fmaf(f, v.w, O.w);
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  const int64_t orow = row * kD + 4 * lane;
+  if (out_f32) {
+    *reinterpret_cast<float4*>(static_cast<float*>(out) + orow) =
+        make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
+  } else {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(O.x * inv, O.y * inv);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(O.z * inv, O.w * inv);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + orow) = pk;
+  }
+}
+
 int max_splits_for(int capacity) {
   const int s = (capacity + 255) / 256;
   return s < 1 ? 1 : (s > 256 ? 256 : s);
 }
 
 }  // namespace
+
+tq_status launch_merge_partials(const float* parts, int n_parts, int64_t rows, void* out,
+                                int out_dtype, cudaStream_t st) {
+  if (rows == 0) return TQ_OK;
+  const int64_t blocks = (rows + 3) / 4;
+  k_merge_partials<<<static_cast<unsigned>(blocks), 128, 0, st>>>(parts, n_parts, rows, out,
+                                                                 out_dtype == TQ_F32);
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ECUDA;
+}
 
 size_t decode_workspace_bytes(int batch, int n_q_heads, int capacity) {
   const size_t parts = static_cast<size_t>(batch) * n_q_heads * max_splits_for(capacity) *
@@ -856,9 +917,10 @@ size_t decode_workspace_bytes(int batch, int n_q_heads, int capacity) {
 
 tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* c, const void* qv, int q_dtype,
                         int n_q_heads, const int32_t* head_map, float sm_scale, void* out,
-                        int out_dtype, float* scores, int64_t scores_ld, void* workspace,
-                        size_t workspace_bytes, cudaStream_t st) {
+                        int out_dtype, float* scores, int64_t scores_ld, float* part_out,
+                        void* workspace, size_t workspace_bytes, cudaStream_t st) {
   DecodeArgs a{};
+  a.part_out = part_out;
   a.k_idx = c->keys.idx;
   a.k_sgn = c->keys.signs;
   a.k_nrm = c->keys.norms;
@@ -904,7 +966,7 @@ tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* c, const void*
 
   int max_len = 0;
   for (int b = 0; b < c->batch; ++b) max_len = c->len_host[b] > max_len ? c->len_host[b] : max_len;
-  if (max_len == 0 && out == nullptr) return TQ_OK;
+  if (max_len == 0 && out == nullptr && part_out == nullptr) return TQ_OK;
 
   // split count: one CTA per SM; minimise waves x (tokens per split + per-CTA set-up) + the
   // final combine (its loads grow with the number of splits). A few SMs are left out of the
@@ -1015,7 +1077,7 @@ tq_status launch_decode_noalloc(const tq_quantizer* q, const tq_kv_cache* c, con
   if (cudaMemsetAsync(static_cast<unsigned char*>(base) + ctr_off, 0, ctr_bytes, st) != cudaSuccess)
     return TQ_ECUDA;
   return launch_decode(q, c, qv, q_dtype, n_q_heads, head_map, sm_scale, out, out_dtype, scores,
-                       scores_ld, base, need, st);
+                       scores_ld, nullptr, base, need, st);
 }
 
 }  // namespace tq

@@ -330,7 +330,35 @@ tq_status tq_decode_attention(const tq_quantizer* q, const tq_kv_cache* c, const
   if (!workspace || !aligned16(workspace)) return TQ_EINVAL;
   if (workspace_bytes < decode_workspace_bytes(c->batch, n_q_heads, c->capacity)) return TQ_EINVAL;
   return launch_decode(q, c, qv, q_dtype, n_q_heads, head_map, sm_scale, out, out_dtype, scores,
-                       scores_ld, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+                       scores_ld, nullptr, workspace, workspace_bytes,
+                       static_cast<cudaStream_t>(stream));
+}
+
+tq_status tq_decode_attention_partial(const tq_quantizer* q, const tq_kv_cache* c, const void* qv,
+                                      int q_dtype, int n_q_heads, const int32_t* head_map,
+                                      float sm_scale, float* part, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  if (!q || !c) return TQ_EINVAL;
+  if (c->value_bits == 0) return TQ_EINVAL;  // a partial carries o: the cache needs values
+  if (!part || !aligned16(part)) return TQ_EINVAL;
+  // every other check is tq_decode_attention's (with a stand-in output pointer)
+  tq_status st = check_decode_args(q, c, qv, q_dtype, n_q_heads, head_map, part, TQ_F32,
+                                   nullptr, 0);
+  if (st != TQ_OK) return st;
+  if (!workspace || !aligned16(workspace)) return TQ_EINVAL;
+  if (workspace_bytes < decode_workspace_bytes(c->batch, n_q_heads, c->capacity)) return TQ_EINVAL;
+  return launch_decode(q, c, qv, q_dtype, n_q_heads, head_map, sm_scale, nullptr, TQ_F32, nullptr,
+                       0, part, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+tq_status tq_merge_partials(const float* parts, int n_parts, int batch, int n_q_heads, void* out,
+                            int out_dtype, void* stream) {
+  if (n_parts < 1 || n_parts > 65536 || batch <= 0 || n_q_heads <= 0 || n_q_heads > 512)
+    return TQ_EINVAL;
+  if (out_dtype != TQ_F32 && out_dtype != TQ_BF16) return TQ_EUNSUPPORTED;
+  if (!parts || !aligned16(parts) || !out || !aligned16(out)) return TQ_EINVAL;
+  return launch_merge_partials(parts, n_parts, static_cast<int64_t>(batch) * n_q_heads, out,
+                               out_dtype, static_cast<cudaStream_t>(stream));
 }
 
 tq_status tq_decode_attention_noalloc(const tq_quantizer* q, const tq_kv_cache* c,

@@ -108,7 +108,9 @@ size_t decode_workspace_bytes(int batch, int n_q_heads, int capacity);
 tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* cache, const void* qv,
                         int q_dtype, int n_q_heads, const int32_t* head_map, float sm_scale,
                         void* out, int out_dtype, float* scores, int64_t scores_ld,
-                        void* workspace, size_t workspace_bytes, cudaStream_t st);
+                        float* part_out, void* workspace, size_t workspace_bytes, cudaStream_t st);
+tq_status launch_merge_partials(const float* parts, int n_parts, int64_t rows, void* out,
+                                int out_dtype, cudaStream_t st);
 
 tq_status launch_decode_noalloc(const tq_quantizer* q, const tq_kv_cache* cache, const void* qv,
                                 int q_dtype, int n_q_heads, const int32_t* head_map,

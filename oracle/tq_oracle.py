@@ -570,6 +570,58 @@ def decode_attention(q: Quantizer, cache: dict, Q: np.ndarray, head_map=None,
     return out, scores
 
 
+# --------------------------------------------------------------------------------------------
+# Context-split decode. Softmax over the union of disjoint token sets is the log-sum-exp merge
+# of per-set results (an identity of the softmax, nothing the pages add): a set's record is
+# m = max_i x_i, l = sum_i 2^(x_i - m), o = sum_i 2^(x_i - m) v_hat_i with the base-2 logits
+# x_i = sm_scale log2(e) s_i of decode_attention; an empty set gives (-inf, 0, 0).
+# --------------------------------------------------------------------------------------------
+def decode_partial(q: Quantizer, cache: dict, Q: np.ndarray, head_map=None,
+                   sm_scale: float | None = None, value_bits: int = 2, group: int = 32):
+    """Records (m (B, H_q), l (B, H_q), o (B, H_q, d)) of this cache's tokens."""
+    Q = np.asarray(Q, dtype=np.float64)
+    B, Hq, d = Q.shape
+    Hkv = cache["k_idx"].shape[1]
+    if head_map is None:
+        head_map = default_head_map(Hq, Hkv)
+    if sm_scale is None or sm_scale == 0.0:
+        sm_scale = 1.0 / math.sqrt(d)
+    m = np.full((B, Hq), -np.inf)
+    l = np.zeros((B, Hq))
+    o = np.zeros((B, Hq, d))
+    for b in range(B):
+        L = int(cache["len"][b])
+        if L == 0:
+            continue
+        for h in range(Hq):
+            kv = head_map[h]
+            planes = dict(idx=cache["k_idx"][b, kv, :L], norms=cache["k_norms"][b, kv, :L])
+            if q.mode == "prod":
+                planes["signs"] = cache["k_signs"][b, kv, :L]
+            v_hat = dequantize_values(cache["v_q"][b, kv, :L], cache["v_params"][b, kv, :L],
+                                      value_bits, d, group)
+            x = key_scores(q, planes, Q[b, h]) * (sm_scale / math.log(2.0))
+            m[b, h] = x.max()
+            w = np.exp2(x - m[b, h])
+            l[b, h] = w.sum()
+            o[b, h] = w @ v_hat
+    return m, l, o
+
+
+def merge_partials(ms, ls, os) -> np.ndarray:
+    """LSE merge of records of disjoint token sets (lists over the sets): sum_r 2^(m_r - M) o_r
+    / sum_r 2^(m_r - M) l_r with M = max_r m_r; zeros where every set is empty."""
+    M = np.max(np.stack(ms), axis=0)
+    Mf = np.where(np.isfinite(M), M, 0.0)
+    num = np.zeros(os[0].shape)
+    den = np.zeros(ls[0].shape)
+    for m, l, o in zip(ms, ls, os):
+        w = np.where(np.isfinite(m), np.exp2(np.where(np.isfinite(m), m, Mf) - Mf), 0.0)
+        num += w[..., None] * o
+        den += w * l
+    return np.where(den[..., None] > 0, num / np.where(den > 0, den, 1.0)[..., None], 0.0)
+
+
 def bf16_rn(x) -> np.ndarray:
     """Round fp64 values to bf16 (RNE) and return them as fp64 (for the bf16 output check)."""
     f = fp32(x)

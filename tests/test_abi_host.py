@@ -103,3 +103,19 @@ def test_selftest_wait_limit_checked_on_host(limit_us):
     with pytest.raises(tq.TQError) as e:
         tq.tq_selftest_bounded_wait(limit_us)
     assert e.value.status == tq.TQ_EINVAL
+
+
+def test_merge_partials_checks_arguments_on_host():
+    """tq_merge_partials rejects bad arguments before any device work (no GPU needed)."""
+    lib = tq._lib
+    buf = (ctypes.c_float * (4 * 132 + 4))()
+    aligned = (ctypes.addressof(buf) + 15) // 16 * 16
+    ok = dict(parts=aligned, n=1, b=1, h=1, out=aligned, dt=tq.TQ_F32)
+    cases = [(dict(n=0), tq.TQ_EINVAL), (dict(n=65537), tq.TQ_EINVAL), (dict(b=0), tq.TQ_EINVAL),
+             (dict(h=513), tq.TQ_EINVAL), (dict(parts=None), tq.TQ_EINVAL),
+             (dict(parts=aligned + 4), tq.TQ_EINVAL), (dict(out=None), tq.TQ_EINVAL),
+             (dict(dt=7), tq.TQ_EUNSUPPORTED)]
+    for change, status in cases:
+        a = dict(ok, **change)
+        assert lib.tq_merge_partials(a["parts"], a["n"], a["b"], a["h"], a["out"], a["dt"],
+                                     None) == status, change

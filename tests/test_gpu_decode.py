@@ -266,3 +266,55 @@ def test_decode_stream_steps():
         ref, _ = O.decode_attention(qo, step_oc, Q[:, heads].astype(np.float64),
                                     head_map=np.zeros(G, dtype=int), value_bits=4)
         check_attention(out[0, heads], ref[0], False)
+
+
+def _slice_oracle_cache(oc, start, stop):
+    out = {k: v[:, :, start:stop] for k, v in oc.items() if k != "len" and v is not None}
+    out["len"] = np.clip(np.asarray(oc["len"]) - start, 0, stop - start)
+    return out
+
+
+@pytest.mark.parametrize("mode,bits,vbits", [("prod", 3, 2), ("mse", 4, 4), ("grouped", 2, 2)])
+def test_decode_context_split_partials_and_merge(mode, bits, vbits):
+    """Context-parallel decode on one GPU: each sequence's context is cut into three ragged
+    slices held by three caches (the shorter sequence leaves the last slice empty).
+    tq_decode_attention_partial on each slice and tq_merge_partials over the three record
+    sets match the oracle's decode over the whole context; each slice's normalised record
+    matches the oracle's attention over that slice; an empty slice gives (-inf, 0, 0); and
+    one slice merged alone reproduces tq_decode_attention bit for bit."""
+    dev = require_cuda()
+    lengths, cap = [1000, 700], 1024
+    if mode == "grouped":
+        qo, qg, oc, cache, Q = grouped_case(120 + bits, 2, 6, 2, lengths, cap, bits, vbits)
+    else:
+        qo, qg, oc, cache, Q = small_case(110 + bits, 2, 6, 2, lengths, cap, bits, vbits, mode)
+    B, Hq = Q.shape[:2]
+    qt = to_device(Q, torch.bfloat16)
+    cuts = (0, 333, 800, 1000)
+    parts = torch.empty((len(cuts) - 1, B, Hq, tq.TQ_PART_FLOATS), device=dev)
+    for i, (a, b) in enumerate(zip(cuts[:-1], cuts[1:])):
+        sl = _slice_oracle_cache(oc, a, b)
+        c = tq.KVCache(qg, B, 2, ((b - a) + 15) // 16 * 16, value_bits=vbits, device=dev)
+        upload_cache(c, sl)
+        ws = tq.alloc_decode_workspace(c, Hq)
+        tq.tq_decode_attention_partial(qg, c, qt, parts[i], ws)
+        torch.cuda.synchronize()
+        rec = parts[i].cpu().numpy().astype(np.float64)
+        m_ref, l_ref, o_ref = O.decode_partial(qo, sl, Q.astype(np.float64), value_bits=vbits)
+        for bb in range(B):
+            if sl["len"][bb] == 0:
+                assert np.all(rec[bb, :, 0] == -np.inf) and np.all(rec[bb, :, 1:] == 0)
+                continue
+            assert np.allclose(rec[bb, :, 0], m_ref[bb], rtol=1e-3, atol=1e-3)
+            check_attention(rec[bb, :, 4:] / rec[bb, :, 1:2], o_ref[bb] / l_ref[bb][:, None], False)
+    out = torch.empty((B, Hq, 128), device=dev)
+    tq.tq_merge_partials(parts, out)
+    ref, _ = O.decode_attention(qo, oc, Q.astype(np.float64), value_bits=vbits)
+    check_attention(out.cpu().numpy(), ref, False)
+    # a single slice: the merge of its one record set is the decode's own output
+    whole = torch.empty((1, B, Hq, tq.TQ_PART_FLOATS), device=dev)
+    ws = tq.alloc_decode_workspace(cache, Hq)
+    tq.tq_decode_attention_partial(qg, cache, qt, whole[0], ws)
+    tq.tq_merge_partials(whole, out)
+    direct, _, _ = run_decode(qg, cache, Q, torch.bfloat16, torch.float32)
+    assert np.array_equal(out.cpu().numpy(), direct)

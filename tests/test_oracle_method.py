@@ -339,3 +339,34 @@ def test_needle_retrieval_small():
             _, sc = O.decode_attention(q, c, needle[None], want_scores=True)
             for h in range(2):
                 assert int(np.argmax(sc[0][h])) == pos
+
+
+def _slice_cache(c, start, stop):
+    """Tokens [start, stop) of every sequence (clipped to its length) as a cache of their own."""
+    out = {k: v[:, :, start:stop] for k, v in c.items() if k != "len"}
+    out["len"] = np.clip(c["len"] - start, 0, stop - start)
+    return out
+
+
+def test_context_split_merge_equals_full_decode():
+    """Softmax over a union of disjoint token sets is the log-sum-exp merge of per-set records:
+    decode_partial over ragged slices of the context (one slice empty for the shorter
+    sequence) merged by merge_partials reproduces decode_attention over the whole context,
+    for prod and mse keys, a GQA head map and a non-default scale."""
+    g = np.random.default_rng(17)
+    for mode, bits in (("prod", 3), ("mse", 2)):
+        q = O.build_quantizer(D, bits, mode, 3)
+        k = g.standard_normal((2, 2, 300, D)) * g.uniform(2, 20, (2, 2, 300, 1))
+        c = _cache_from(q, k, g.standard_normal((2, 2, 300, D)))
+        c["len"] = np.array([300, 120])
+        Q = g.standard_normal((2, 4, D))
+        hm = np.array([0, 1, 1, 0])
+        full, _ = O.decode_attention(q, c, Q, head_map=hm, sm_scale=0.07)
+        for cuts in ((0, 300), (0, 100, 300), (0, 37, 150, 299, 300)):
+            parts = [O.decode_partial(q, _slice_cache(c, a, b), Q, head_map=hm, sm_scale=0.07)
+                     for a, b in zip(cuts[:-1], cuts[1:])]
+            merged = O.merge_partials(*zip(*parts))
+            assert np.allclose(merged, full, rtol=0, atol=1e-12), (mode, cuts)
+        # an empty slice: (-inf, 0, 0), and merging it changes nothing
+        m, l, o = O.decode_partial(q, _slice_cache(c, 300, 300), Q, head_map=hm)
+        assert np.all(m == -np.inf) and np.all(l == 0) and np.all(o == 0)
