@@ -297,7 +297,6 @@ __global__ void __launch_bounds__(128, 2)
       dcsP2[t] = pk2(ncs[NL / 2 + t + 1] - ncs[NL / 2 + t], ncs[NL / 2 + t + 1] - ncs[NL / 2 + t]);
     }
     const uint64_t ncsP02 = pk2(ncs[NL / 2], ncs[NL / 2]);
-    const uint64_t kSplit2 = pk2(8192.f, 8192.f);  // c = 8192 r + r
 
     uint64_t racc[4];
 #pragma unroll
@@ -353,13 +352,14 @@ __global__ void __launch_bounds__(128, 2)
           if constexpr (!PROD) continue;
           const uint64_t r = SYM ? fma2(sg2, c2, mul2(y2, scl2)) : fma2(y2, scl2, c2);
           racc[pi & 3] = fma2(r, r, racc[pi & 3]);
-          // Veltkamp split: hi keeps the top 11 significant bits (exact in fp16 for |r| < 2^15),
-          // lo = r - hi exactly (13 bits, rounded to fp16's 11). c = RN(8193 r) comes from one
-          // fma so that no multiply is left for the compiler to fuse with the next subtraction.
-          const uint64_t cc = fma2(r, kSplit2, r);
-          const uint64_t hi = sub2(cc, sub2(cc, r));
-          const float2 hv = up2(hi), lv = up2(sub2(r, hi));
-          hw[pi] = h2_bits(hv.x, hv.y);
+          // hi/lo split: hi = r with its 13 low mantissa bits cleared (11 significant bits,
+          // exact in fp16 for |r| < 2^15), lo = r - hi exactly in fp32 (at most 13 significant
+          // bits, rounded to fp16's 11): |r - hi16 - lo16| <= 2^-21 |r|
+          const float2 rv = up2(r);
+          const float hx = __uint_as_float(__float_as_uint(rv.x) & 0xffffe000u);
+          const float hy = __uint_as_float(__float_as_uint(rv.y) & 0xffffe000u);
+          const float2 lv = up2(sub2(r, pk2(hx, hy)));
+          hw[pi] = h2_bits(hx, hy);
           lw[pi] = h2_bits(lv.x, lv.y);
         }
       }
