@@ -23,10 +23,11 @@
 // (chunk w, w + 16, ... of the range), so no CTA-wide barrier sits in the loop: each lane
 // holds its token's key bytes in registers (prefetched one chunk ahead), scores it from the
 // tables, and the warp runs the online softmax; the chunk's value bytes arrive in the warp's
-// own shared-memory slot by cp.async, and for P.V the lanes split the 128 channels (4 per
-// lane, one token a step) with packed fp32x2 FMAs. Each CTA merges its warps and writes a
-// partial (m, l, o); the last CTA of a (sequence, head group) to finish merges all partials
-// (an atomic counter, no waiting).
+// own shared-memory slot by cp.async, and for P.V each half-warp takes one token a step with
+// its 16 lanes splitting the 128 channels (8 per lane) in packed fp32x2 FMAs. Each CTA merges
+// its warps and writes a partial (m, l, o); the last CTA of a (sequence, head group) to finish
+// merges all partials (an atomic counter, no waiting), or writes the merged partial itself
+// for a context-parallel decode.
 #include <cfloat>
 #include <cmath>
 #include <mutex>
