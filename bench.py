@@ -321,10 +321,12 @@ def run_tq(args):
                   "KV head + decode)",
         "value": value, "unit": "keys/s", "n_gpus": world, "steps": steps, "warmup": warm,
         "ms_per_step": tot_ms_max / steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in; u8 packed; fp32 accum",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded torch CUDA generator; N(0,1) x U[2,20] keys)",
         "config": {"workload": wl_desc,
                    "global_batch": B * world, "seq_len": N, "parallelism": f"replicas x{world}",
+                   "data_types": "bf16 query and new K/V rows, u8 packed cache, fp16 norms "
+                                 "and value params, fp32 arithmetic",
                    "l2": "flushed (256 MiB write) before each step, outside its events"},
         "decode_gbs": achieved,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
