@@ -301,8 +301,8 @@ __global__ void __launch_bounds__(128, 2)
     uint64_t racc[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) racc[i] = pk2(0.f, 0.f);
-#pragma unroll 1
-    for (int g = 0; g < NG; ++g) {
+    // decisions of column group g (pairs [GP g, GP g + GP)) from its TMEM columns yg
+    auto decide_group = [&](int g, const uint32_t (&yg)[GP / 8][16]) {
       // index words of elements [GP g, GP g + GP) (.x) and +64 (.y), accumulated in fp32 as
       // exact integers: codes of pairs [0, GP/2) in wa, [GP/2, GP) in wb (each < 2^16)
       // symmetric path: each word starts at sum_j kw_j (L - 1)/2 over its pairs
@@ -311,8 +311,7 @@ __global__ void __launch_bounds__(128, 2)
       uint32_t hw[GP], lw[GP];
 #pragma unroll
       for (int q = 0; q < GP / 8; ++q) {
-        uint32_t yv[16];
-        tmem_ld16_sync(tlane + 2 * GP * g + 16 * q, yv);
+        const uint32_t (&yv)[16] = yg[q];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int pi = 8 * q + i;  // pair index within the group
@@ -383,6 +382,41 @@ __global__ void __launch_bounds__(128, 2)
                                  ((__float_as_uint(fb.x) & 0xffffu) << kHalfBits);
         sCode[(NG + g) * kTile + tid] = (__float_as_uint(fa.y) & 0xffffu) |
                                         ((__float_as_uint(fb.y) & 0xffffu) << kHalfBits);
+      }
+    };
+    // The loads of group g + 1 are issued before group g's decisions and waited for after
+    // them, so the TMEM latency overlaps the work (NG is even).
+    auto issue = [&](int g, uint32_t (&yg)[GP / 8][16]) {
+#pragma unroll
+      for (int q = 0; q < GP / 8; ++q) tmem_ld16(tlane + 2 * GP * g + 16 * q, yg[q]);
+    };
+    auto tie = [&](uint32_t (&yg)[GP / 8][16]) {
+#pragma unroll
+      for (int q = 0; q < GP / 8; ++q) tmem_ld_wait_tied16(yg[q]);
+    };
+    // (prod with 1- or 2-bit indices keeps one group in flight: a second buffer would spill)
+    constexpr bool kAhead = !(PROD && MB <= 2);
+    static_assert(NG % 2 == 0, "column groups come in pairs");
+    uint32_t yA[GP / 8][16];
+    if constexpr (kAhead) {
+      uint32_t yB[GP / 8][16];
+      issue(0, yA);
+      tie(yA);
+#pragma unroll 1
+      for (int g = 0; g < NG; g += 2) {
+        issue(g + 1, yB);
+        decide_group(g, yA);
+        tie(yB);
+        if (g + 2 < NG) issue(g + 2, yA);
+        decide_group(g + 1, yB);
+        if (g + 2 < NG) tie(yA);
+      }
+    } else {
+#pragma unroll 1
+      for (int g = 0; g < NG; ++g) {
+        issue(g, yA);
+        tie(yA);
+        decide_group(g, yA);
       }
     }
     const float2 r2 = up2(add2(add2(racc[0], racc[1]), add2(racc[2], racc[3])));
@@ -680,17 +714,24 @@ __global__ void __launch_bounds__(128, 2)
     for (int t = 0; t < NTO; ++t) TO[t] = n_o > 0.f ? thrO[t] * n_o : thrO[t];
 #pragma unroll
     for (int t = 0; t < NTN; ++t) TN[t] = n_n > 0.f ? thrN[t] * ns : thrN[t];
+    // the next unit's columns are loaded while the current unit is decided
+    uint32_t yA[16], yB[16];
+    tmem_ld16(tlane, yA);
+    tmem_ld_wait_tied16(yA);
+    tmem_ld16(tlane + 16, yB);
+    decide16<WO, NTO>(yA, TO, sCode, 0, tid);
+    tmem_ld_wait_tied16(yB);
+    tmem_ld16(tlane + 32, yA);
+    decide16<WO, NTO>(yB, TO, sCode, WO, tid);
+    tmem_ld_wait_tied16(yA);
 #pragma unroll 1
-    for (int u = 0; u < 2; ++u) {
-      uint32_t yv[16];
-      tmem_ld16_sync(tlane + 16 * u, yv);
-      decide16<WO, NTO>(yv, TO, sCode, u * WO, tid);
-    }
-#pragma unroll 1
-    for (int u = 0; u < 6; ++u) {
-      uint32_t yv[16];
-      tmem_ld16_sync(tlane + 32 + 16 * u, yv);
-      decide16<WN, NTN>(yv, TN, sCode, HWO + u * WN, tid);
+    for (int u = 0; u < 6; u += 2) {
+      tmem_ld16(tlane + 32 + 16 * (u + 1), yB);
+      decide16<WN, NTN>(yA, TN, sCode, HWO + u * WN, tid);
+      tmem_ld_wait_tied16(yB);
+      if (u + 2 < 6) tmem_ld16(tlane + 32 + 16 * (u + 2), yA);
+      decide16<WN, NTN>(yB, TN, sCode, HWO + (u + 1) * WN, tid);
+      if (u + 2 < 6) tmem_ld_wait_tied16(yA);
     }
 
     if (valid) {

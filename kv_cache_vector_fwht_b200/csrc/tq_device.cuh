@@ -289,6 +289,16 @@ __device__ __forceinline__ void tmem_ld16_sync(uint32_t taddr, uint32_t (&r)[16]
                :
                : "memory");
 }
+// tcgen05.wait::ld tied to the registers of an earlier tmem_ld16, for loads issued ahead of
+// the work they overlap (the wait covers every load this thread has issued).
+__device__ __forceinline__ void tmem_ld_wait_tied16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
 __device__ __forceinline__ void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32]) {
   tmem_ld32(taddr, r);
   asm volatile("tcgen05.wait::ld.sync.aligned;\n"
