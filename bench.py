@@ -307,9 +307,16 @@ def run_tq(args):
     e2e_ms_max = max_over_ranks(e2e_ms, world)
     e2e_value = sum_over_ranks(e2e_keys, world) / (e2e_ms_max / 1e3) if e2e_steps else None
 
+    # the block shape the library picks (tq.h, tq_set_decode_policy): up to 8 query heads per
+    # block (two table sets) when a KV head has more than 4 and there are >= 4 x 384 (token,
+    # KV head) units per SM (all SMs but 4), else up to 4
     heads_per_kv = Hq // Hkv
-    nh_cta = -(-heads_per_kv // -(-heads_per_kv // 4))     # query heads per CTA (groups of <= 4)
-    nh_tpl = 2 if nh_cta <= 2 else nh_cta
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    two_sets = heads_per_kv > 4 and B * Hkv * N >= 4 * 384 * max(1, n_sms - 4)
+    cap = 8 if two_sets else 4
+    nh_cta = -(-heads_per_kv // -(-heads_per_kv // cap))   # query heads per block
+    nh_tpl = (2 if nh_cta <= 2 else nh_cta) if not two_sets else (6 if nh_cta <= 6 else 8)
+    n_sets = 2 if two_sets else 1
     wl_desc = {"decode-s": "decode-s: batch 1, 12 q heads / 2 kv heads, d 128, ctx 32768, "
                            "keys 3-bit prod, values 2-bit g32",
                "decode-l": "decode-l: batch 8, 28 q heads / 4 kv heads, d 128, ctx 32768, "
@@ -331,7 +338,8 @@ def run_tq(args):
         "decode_gbs": achieved,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": None,
-                     "kernel": f"k_decode<{WL['key_bits'] - 1},{WL['value_bits']},{nh_tpl}>",
+                     "kernel": f"k_decode<{WL['key_bits'] - 1},{WL['value_bits']},{nh_tpl},prod,"
+                               f"{n_sets} table set{'s' if n_sets > 1 else ''}>",
                      "bytes_per_launch": dec_bytes, "avg_launch_us": dec_avg_ms * 1e3,
                      "peak_kind": f"{peak_kind} (hbm_gbs, burst)"},
         "e2e": {"value": e2e_value, "unit": "keys/s", "h2d_bytes_per_step": int(

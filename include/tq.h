@@ -230,7 +230,21 @@ tq_status tq_decode_attention_noalloc(const tq_quantizer* q, const tq_kv_cache* 
                                       void* out_dev, int out_dtype,
                                       float* scores_dev, int64_t scores_ld, void* stream);
 
-/* ---- context-parallel decode (a cache's context split into slices, e.g. one per GPU) ----
+/* Shape of the fused decode's thread blocks (process-wide; a tuning and testing knob, the
+ * results do not depend on it beyond fp32 rounding order). A block scores and sums the
+ * tokens of one KV head for a group of its query heads. TQ_DECODE_AUTO (the default): groups
+ * of up to 8 query heads (two 4-head lookup-table sets, 12 warps) when a KV head has more
+ * than 4 and the decode holds at least 4 x 384 (token, KV head) units per SM, else groups of
+ * up to 4 (one table set, 16 warps). TQ_DECODE_ONE_SET and TQ_DECODE_TWO_SETS force one
+ * shape (two sets only where a KV head has more than 4 query heads and the two-set tables
+ * fit the shared memory; grouped keys always use one set). Writes the previous policy to
+ * `previous` (nullable); TQ_EINVAL for another value (nothing changed). */
+#define TQ_DECODE_AUTO 0
+#define TQ_DECODE_ONE_SET 1
+#define TQ_DECODE_TWO_SETS 2
+tq_status tq_set_decode_policy(int policy, int* previous);
+
+/* ---- context-parallel decode/* ---- context-parallel decode (a cache's context split into slices, e.g. one per GPU) ----
  * Softmax attention over the union of the slices equals the LSE merge of per-slice partial
  * results (the merge the fused decode kernel already runs between its own context splits):
  *   step 1, per slice:  tq_decode_attention_partial -> (m, l, o) per (sequence, query head)

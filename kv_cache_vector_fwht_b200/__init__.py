@@ -30,7 +30,7 @@ D = 128
 EXPORTED = ["tq_build_codebook", "tq_free", "tq_key_layout", "tq_host_tables",
             "tq_quantize_keys", "tq_dequantize_keys", "tq_quantize_values", "tq_append", "tq_decode_workspace_bytes",
             "tq_decode_attention", "tq_decode_attention_noalloc", "tq_decode_attention_partial",
-            "tq_merge_partials", "tq_sync_status",
+            "tq_merge_partials", "tq_set_decode_policy", "tq_sync_status",
             "tq_selftest_bounded_wait", "tq_status_string", "tq_abi_version"]
 
 
@@ -93,6 +93,8 @@ _lib.tq_decode_attention_partial.argtypes = [c_void_p, POINTER(KVCacheDesc), c_v
 _lib.tq_decode_attention_partial.restype = c_int
 _lib.tq_merge_partials.argtypes = [c_void_p, c_int, c_int, c_int, c_void_p, c_int, c_void_p]
 _lib.tq_merge_partials.restype = c_int
+_lib.tq_set_decode_policy.argtypes = [c_int, POINTER(c_int)]
+_lib.tq_set_decode_policy.restype = c_int
 _lib.tq_status_string.argtypes = [c_int]
 _lib.tq_status_string.restype = ctypes.c_char_p
 _lib.tq_abi_version.argtypes = []
@@ -340,6 +342,16 @@ def tq_decode_attention(q: Quantizer, cache: KVCache, query, out=None, workspace
                                     _dtype_code(out) if out is not None else TQ_F32,
                                     _ptr(scores), sld, _ptr(workspace), wbytes, _stream(stream)),
            "tq_decode_attention")
+
+
+TQ_DECODE_AUTO, TQ_DECODE_ONE_SET, TQ_DECODE_TWO_SETS = 0, 1, 2
+
+
+def tq_set_decode_policy(policy: int) -> int:
+    """Process-wide decode block shape (see tq.h); returns the previous policy."""
+    prev = c_int(0)
+    _check(_lib.tq_set_decode_policy(int(policy), ctypes.byref(prev)), "tq_set_decode_policy")
+    return prev.value
 
 
 TQ_PART_FLOATS = 132   # floats per partial record: m, l, 0, 0, o[128]

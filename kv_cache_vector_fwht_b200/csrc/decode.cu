@@ -28,6 +28,7 @@
 // its warps and writes a partial (m, l, o); the last CTA of a (sequence, head group) to finish
 // merges all partials (an atomic counter, no waiting), or writes the merged partial itself
 // for a context-parallel decode.
+#include <atomic>
 #include <cfloat>
 #include <cmath>
 #include <mutex>
@@ -38,11 +39,10 @@
 namespace tq {
 namespace {
 
-constexpr int kMaxHeads = 4;      // query heads per CTA (one 16-byte table entry)
+constexpr int kMaxHeads = 4;      // query heads of one table set (one 16-byte table entry)
+constexpr int kMaxSlots = 8;      // query heads per CTA: at most two table sets
 constexpr int kMaxGroups = 256;
-constexpr int kThreads = 512;
-constexpr int kWarps = kThreads / 32;
-constexpr int kChunkStride = 32 * kWarps;  // tokens between a warp's consecutive chunks
+std::atomic<int> g_decode_policy{TQ_DECODE_AUTO};
 constexpr int kPartStride = 132;  // floats per (head, split) partial: m, l, pad, o[128]
 constexpr int kSrotStride = 272;  // bytes per staged q half row (256 + 16: bank spread)
 // dequant pairs of a warp: [group][token] float4 rows of 34 entries, so that the 4 groups x 2
@@ -70,7 +70,7 @@ struct DecodeArgs {
   int max_len;  // host copy of the longest sequence (an upper bound of every len[b])
   float scale_log2, inv_scale_log2;
   int16_t g_kv[kMaxGroups];
-  int16_t g_heads[kMaxGroups][kMaxHeads];
+  int16_t g_heads[kMaxGroups][kMaxSlots];
   int8_t g_n[kMaxGroups];
 };
 
@@ -90,12 +90,23 @@ __device__ __forceinline__ uint64_t sign_pair(int mask) {
 // 32-channel outlier group at b + 1 bits and a 96-channel group at b bits, one norm each).
 enum KeyKind { kMse = 0, kProd = 1, kGrp = 2 };
 
+// CTA shape for NSET table sets of 4 head slots: 16 warps with one set, 12 with two (whose
+// tables and per-head state take more of the shared memory and registers).
+template <int NSET>
+struct Cfg {
+  static constexpr int slots = kMaxHeads * NSET;            // head slots
+  static constexpr int threads = NSET == 1 ? 512 : 384;
+  static constexpr int warps = threads / 32;
+  static constexpr int chunk_stride = 32 * warps;           // tokens between a warp's chunks
+};
+
 // Shared-memory plan. MB: index bits (mse, prod) or the grouped base bits b. A token's key
 // bytes form two lookup segments: I (index bytes; grouped: the outlier group) and S (prod:
 // the QJL sign bytes; grouped: the normal group, padded with zero bytes to whole 8-byte
 // blocks). Each segment accumulates its own sum; the two norms scale them.
-template <int MB, int VB, int K>
+template <int MB, int VB, int K, int NSET>
 struct Lay {
+  static constexpr int SL = Cfg<NSET>::slots, kWarps = Cfg<NSET>::warps;
   static constexpr bool GRP = K == kGrp;
   static constexpr int MI = GRP ? MB + 1 : MB;                     // segment I code bits
   static constexpr int MS = GRP ? MB : 1;                          // segment S code bits
@@ -110,11 +121,17 @@ struct Lay {
   static constexpr int NB = K == kMse ? 2 : 4;                     // norm bytes per token
   static constexpr int VQB = VB ? kD * VB / 8 : 0;         // value code bytes per token
   static constexpr int VPB = VB ? 16 : 0;                  // value params per token
+  // Tables: NSET sets (head slots 4s .. 4s + 3), each set contiguous. With two sets the
+  // QJL sign tables are nibble tables (16 entries x 32 nibble positions, no mirror), which
+  // keeps two sets of 3-bit prod tables within the shared memory.
+  static constexpr bool NIB = K == kProd && NSET == 2;
+  static constexpr int SETI = EI * PI * 16;                          // bytes of one index set
+  static constexpr int SETS = NIB ? 16 * 32 * 16 : ES * PS * 16;     // bytes of one sign set
   static constexpr int lutI = 0;
-  static constexpr int lutS = lutI + EI * PI * 16;
-  static constexpr int qrT = lutS + ES * PS * 16;                    // q_rot [128][4] f32
-  static constexpr int sqT = qrT + kD * kMaxHeads * 4;               // Sq    [128][4] f32
-  static constexpr int qhi = sqT + kD * kMaxHeads * 4;               // hi [8][136] f16
+  static constexpr int lutS = lutI + NSET * SETI;
+  static constexpr int qrT = lutS + NSET * SETS;                     // q_rot [128][SL] f32
+  static constexpr int sqT = qrT + kD * SL * 4;               // Sq    [128][SL] f32
+  static constexpr int qhi = sqT + kD * SL * 4;               // hi [8][136] f16
   static constexpr int qlo = qhi + 8 * kSrotStride;                  // lo [8][136] f16
   static constexpr int qinv = qlo + 8 * kSrotStride;                 // [8] f32
   // per-warp slots: value bytes of the chunk, p pairs, dequant pairs
@@ -123,26 +140,36 @@ struct Lay {
   static constexpr int o_vq = 0;                 // within a warp's value slot
   static constexpr int o_vp = 32 * VQB;
   static_assert(o_vq == 0 && o_vp >= 0, "value slot layout");
-  static constexpr int ppair = wv + kWarps * wv_bytes;                 // [warp][2][32] 2x(p, p)
-  static constexpr int vpair = ppair + kWarps * 32 * kMaxHeads * 8;    // [warp][4][34] f32x4
+  static constexpr int ppair = wv + kWarps * wv_bytes;                 // [warp][32][SL] (p, p) pairs
+  static constexpr int vpair = ppair + kWarps * 32 * SL * 8;    // [warp][4][34] f32x4
   static constexpr int end_v = vpair + (VB ? kWarps * 4 * kVpStride * 16 : 0);
-  static constexpr int merge = kWarps * kMaxHeads * kPartStride * 4;   // reuses wv..
+  static constexpr int merge = kWarps * SL * kPartStride * 4;   // reuses wv..
   // prologue scratch for the nibble partial tables (the value slots may be filling then)
   static constexpr int PNI = MI == 3 ? 0 : PI;                         // nibble-built positions
   static constexpr int PNS = MS == 3 ? 0 : PS;
   static constexpr int scratch = VB ? ppair : wv;
-  static constexpr int scratch_bytes = (2 * 16 * PNI + 2 * 16 * PNS) * 16;
-  static constexpr int total = (end_v - wv) >= merge ? end_v : wv + merge;
+  static constexpr int scratch_bytes = NSET * (2 * 16 * PNI + (NIB ? 0 : 2 * 16 * PNS)) * 16;
+  // the last CTA's merge: split maxima, sums and weights per head slot, 4 SL floats, and
+  // (slice, active head) partial sums (at most one slice of 32 float4 per warp)
+  static constexpr int last = 3 * SL * 256 * 4 + 4 * SL * 4 + kWarps * 32 * 16;
+  static constexpr int need_wv = merge > last ? merge : last;
+  static constexpr int total0 = (end_v - wv) >= need_wv ? end_v : wv + need_wv;
+  static constexpr int total = total0 >= scratch + scratch_bytes ? total0 : scratch + scratch_bytes;
   static_assert(IBI % 8 == 0 && PS % 8 == 0, "whole 8-byte lookup blocks");
-  static_assert(scratch + scratch_bytes <= total, "prologue scratch fits");
-  static_assert(total <= 227 * 1024, "decode shared memory budget");
+  static_assert(NSET == 1 || K != kGrp, "grouped keys use one table set");
+  static constexpr bool fits = total <= 227 * 1024;                  // decode shared memory budget
 };
 
-// Accumulate one 4-head table entry with sign: acc[j] += sg * entry.
-__device__ __forceinline__ void lut_acc(uint64_t (&acc)[2], const uint8_t* p, uint64_t sg) {
-  const ulonglong2 L = *reinterpret_cast<const ulonglong2*>(p);
-  acc[0] = fma2(sg, L.x, acc[0]);
-  acc[1] = fma2(sg, L.y, acc[1]);
+// Accumulate one 4-head table entry of each of the NS table sets (SETB bytes apart) with
+// sign: acc[s][j] += sg * entry_s.
+template <int NS, int SETB>
+__device__ __forceinline__ void lut_acc(uint64_t (&acc)[NS][2], const uint8_t* p, uint64_t sg) {
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    const ulonglong2 L = *reinterpret_cast<const ulonglong2*>(p + s * SETB);
+    acc[s][0] = fma2(sg, L.x, acc[s][0]);
+    acc[s][1] = fma2(sg, L.y, acc[s][1]);
+  }
 }
 
 // Byte k of w sign-extended to 32 bits (prmt: a selector nibble with its top bit set
@@ -163,10 +190,10 @@ __device__ __forceinline__ void rot_block(uint32_t w0, uint32_t w1, bool swap, u
   out1 = __funnelshift_r(b, a, sh);
 }
 
-// Lookups of one 8-byte block of mirror-symmetric bytes (index bytes of 1- or 2-bit codes,
-// or sign bytes): byte i of the rotated block is position 8 blk + ((l + i) mod 8).
-template <int ROWB>
-__device__ __forceinline__ void block_lookups(uint64_t (&acc)[2], uint32_t R0, uint32_t R1,
+// Lookups of one 8-byte block of mirror-symmetric bytes (index bytes of 1-, 2- or 4-bit
+// codes, or sign bytes): byte i of the rotated block is position 8 blk + ((l + i) mod 8).
+template <int ROWB, int NS, int SETB>
+__device__ __forceinline__ void block_lookups(uint64_t (&acc)[NS][2], uint32_t R0, uint32_t R1,
                                               const uint8_t* tab, int blk,
                                               const uint32_t (&rot16)[8]) {
 #pragma unroll
@@ -175,16 +202,15 @@ __device__ __forceinline__ void block_lookups(uint64_t (&acc)[2], uint32_t R0, u
     const int sx = byte_sx(R, i & 3);
     const int msk = sx >> 31;
     const uint32_t e = static_cast<uint32_t>(sx ^ msk);  // canonical entry, 0..127
-    const uint8_t* p = tab + 128 * blk + e * ROWB + rot16[i];
-    lut_acc(acc, p, sign_pair(msk));
+    lut_acc<NS, SETB>(acc, tab + 128 * blk + e * ROWB + rot16[i], sign_pair(msk));
   }
 }
 
 // Lookups of one 8-byte block of bytes holding two 3-bit codes in their nibbles: the mirror
 // flips both codes (k -> 7 - k), chosen by bit 6 (high code >= 4); entry = low code + 8 (high
 // code mod 4).
-template <int ROWB>
-__device__ __forceinline__ void block_lookups3(uint64_t (&acc)[2], uint32_t R0, uint32_t R1,
+template <int ROWB, int NS, int SETB>
+__device__ __forceinline__ void block_lookups3(uint64_t (&acc)[NS][2], uint32_t R0, uint32_t R1,
                                                const uint8_t* tab, int blk,
                                                const uint32_t (&rot16)[8]) {
 #pragma unroll
@@ -193,33 +219,61 @@ __device__ __forceinline__ void block_lookups3(uint64_t (&acc)[2], uint32_t R0, 
     const int msk = static_cast<int>(v << 25) >> 31;
     const uint32_t vc = v ^ (static_cast<uint32_t>(msk) & 0x77u);
     const uint32_t en = (vc & 7u) | ((vc >> 1) & 0x18u);
-    lut_acc(acc, tab + 128 * blk + en * ROWB + rot16[i], sign_pair(msk));
+    lut_acc<NS, SETB>(acc, tab + 128 * blk + en * ROWB + rot16[i], sign_pair(msk));
   }
 }
 
 // Segment lookups over 8-byte blocks of words w (2 words a block).
-template <int MBITS, int NPOS>
-__device__ __forceinline__ void segment_lookups(uint64_t (&acc)[2], const uint32_t* w,
+template <int MBITS, int NPOS, int NS, int SETB>
+__device__ __forceinline__ void segment_lookups(uint64_t (&acc)[NS][2], const uint32_t* w,
                                                 const uint8_t* tab, bool swap, uint32_t sh,
                                                 const uint32_t (&rot16)[8]) {
 #pragma unroll
   for (int blk = 0; blk < NPOS / 8; ++blk) {
     uint32_t R0, R1;
     rot_block(w[2 * blk], w[2 * blk + 1], swap, sh, R0, R1);
-    if constexpr (MBITS == 3) block_lookups3<NPOS * 16>(acc, R0, R1, tab, blk, rot16);
-    else block_lookups<NPOS * 16>(acc, R0, R1, tab, blk, rot16);
+    if constexpr (MBITS == 3) block_lookups3<NPOS * 16, NS, SETB>(acc, R0, R1, tab, blk, rot16);
+    else block_lookups<NPOS * 16, NS, SETB>(acc, R0, R1, tab, blk, rot16);
+  }
+}
+
+// QJL sign lookups from nibble tables (16 entries x 32 nibble positions, entry e of position
+// p at (e 32 + p) 16 bytes): the 128 sign bits as 32 nibbles. Each 32-bit word (8 nibble
+// positions) is rotated by this lane's 4 (l mod 8) bits, so that at step i lane l reads
+// position 8 blk + ((l + i) mod 8) and the eight lanes of a 16-byte phase fall in eight
+// different bank groups.
+template <int NS, int SETB>
+__device__ __forceinline__ void nibble_lookups(uint64_t (&acc)[NS][2], const uint32_t (&w)[4],
+                                               const uint8_t* tab, uint32_t r8,
+                                               const uint32_t (&rot16)[8]) {
+#pragma unroll
+  for (int blk = 0; blk < 4; ++blk) {
+    const uint32_t rot = __funnelshift_r(w[blk], w[blk], 4 * r8);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint8_t* p = tab + ((rot >> (4 * i)) & 15u) * 512 + blk * 128 + rot16[i];
+#pragma unroll
+      for (int s = 0; s < NS; ++s) {
+        const ulonglong2 L = *reinterpret_cast<const ulonglong2*>(p + s * SETB);
+        acc[s][0] = add2(acc[s][0], L.x);
+        acc[s][1] = add2(acc[s][1], L.y);
+      }
+    }
   }
 }
 
 // K = kMse: s = n16 <Pi q, c[idx]>; kProd: + r16 sqrt(pi/2)/d <S q, 2 sigma - 1>;
 // kGrp: s = n_o <Pi_o q_o, c_o[idx_o]> + n_n <Pi_n q_n, c_n[idx_n]> over the two channel
 // groups (Pi_g: 32-point Hadamard blocks after the group's signs).
-template <int MB, int VB, int NH, int K>
-__global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ DecodeArgs a) {
-  using Lo = Lay<MB, VB, K>;
+template <int MB, int VB, int NH, int K, int NSET>
+__global__ void __launch_bounds__(Cfg<NSET>::threads, 1) k_decode(const __grid_constant__ DecodeArgs a) {
+  using Lo = Lay<MB, VB, K, NSET>;
+  constexpr int NT = Cfg<NSET>::threads, NWp = Cfg<NSET>::warps, CS = Cfg<NSET>::chunk_stride;
+  constexpr int SL = Cfg<NSET>::slots;
   constexpr bool PROD = K == kProd, GRP = K == kGrp, TWO = K != kMse;
   constexpr int IB = Lo::IB, PI = Lo::PI, KW = Lo::KW;
-  static_assert(NH >= 1 && NH <= kMaxHeads, "heads per CTA");
+  static_assert(NH >= 1 && NH <= SL, "heads per CTA");
+  static_assert(Lo::fits, "decode shared memory budget");
   constexpr bool HAS_V = VB != 0;
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* lutI = smem + Lo::lutI;
@@ -238,16 +292,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
   const int t0 = split * a.tokens_per_split;
   const int64_t kvrow = (static_cast<int64_t>(b) * a.n_kv_heads + kv) * a.capacity;
 
-  // P.V: half-warp hw = lane / 16 takes every other token of a chunk; lane owns channels
-  // 8 j16 .. 8 j16 + 7 (j16 = lane mod 16) as four fp32 pairs
+  // P.V, one table set: half-warp hw = lane / 16 takes every other token of a chunk and lane
+  // owns channels 8 j16 .. 8 j16 + 7 (j16 = lane mod 16) as four fp32 pairs; two sets (up to 8
+  // heads, whose accumulators would not fit twice): the warp takes one token a step and lane
+  // owns channels 4 lane .. 4 lane + 3 as two pairs.
+  constexpr int OC = NSET == 1 ? 4 : 2;
   float m[NH], l[NH];
-  uint64_t o[NH][4];
+  uint64_t o[NH][OC];
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
     m[h] = -INFINITY;
     l[h] = 0.f;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) o[h][k] = 0ull;
+    for (int k = 0; k < OC; ++k) o[h][k] = 0ull;
   }
 
   // The prologue reads only the query and the quantizer's tables, so it runs before the
@@ -267,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
       const int len_b[5] = {n * IB, PROD ? n * 16 : 0, n * Lo::NB, n * Lo::VQB, VB ? n * 16 : 0};
 #pragma unroll
       for (int r = 0; r < 5; ++r)
-        for (int off = threadIdx.x * 128; off < len_b[r]; off += kThreads * 128)
+        for (int off = threadIdx.x * 128; off < len_b[r]; off += NT * 128)
           asm volatile("prefetch.global.L2 [%0];" ::"l"(rng[r] + off));
     }
     // key bytes of this lane's token in chunk c (zeros past the range)
@@ -385,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int j = 4 * lane + i;
-        if (warp < kMaxHeads) qrT[j * kMaxHeads + warp] = v[i];
+        if (warp < SL) qrT[j * SL + warp] = v[i];
         const float sv = v[i] * scl;
         const __half hi = __float2half_rn(sv);
         const __half lo = __float2half_rn(sv - __half2float(hi));
@@ -415,14 +472,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
               : "r"(afr[kk][0]), "r"(afr[kk][1]), "r"(afr[kk][2]), "r"(afr[kk][3]), "r"(b0), "r"(b1));
         }
       }
-      if (2 * t < kMaxHeads) {  // columns 2t, 2t + 1 are head slots 0..3
+      if (2 * t < SL) {  // columns 2t, 2t + 1 are head slots
         const float s0 = qinv[2 * t] * 0.088388347648318440550f;      // / sqrt(128)
         const float s1 = qinv[2 * t + 1] * 0.088388347648318440550f;
         const int j0 = 16 * warp + g;
-        sqT[j0 * kMaxHeads + 2 * t] = c0 * s0;
-        sqT[j0 * kMaxHeads + 2 * t + 1] = c1 * s1;
-        sqT[(j0 + 8) * kMaxHeads + 2 * t] = c2 * s0;
-        sqT[(j0 + 8) * kMaxHeads + 2 * t + 1] = c3 * s1;
+        sqT[j0 * SL + 2 * t] = c0 * s0;
+        sqT[j0 * SL + 2 * t + 1] = c1 * s1;
+        sqT[(j0 + 8) * SL + 2 * t] = c2 * s0;
+        sqT[(j0 + 8) * SL + 2 * t + 1] = c3 * s1;
       }
     }
     __syncthreads();
@@ -444,58 +501,78 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
                            : a.scale_log2 * 1.2533141373155002512f / 128.f;
       // Entries of 1-, 2- and 4-bit code bytes and of sign bytes are sums of two nibble
       // partials (low and high half of the byte): NI[half][n][p] and NS[half][n][p]
-      // (16-byte float4 of the 4 head slots) are built in a scratch region first; entry
-      // (e, p) = N[0][e mod 16][p] + N[1][e / 16][p].
+      // (16-byte float4 of a set's 4 head slots) are built in a scratch region first; entry
+      // (e, p) = N[0][e mod 16][p] + N[1][e / 16][p]. Table set s holds head slots 4s .. 4s + 3
+      // (column 4s of the [128][SL] q_rot and Sq arrays).
+      constexpr int NIS = 2 * 16 * PNI, NSS = Lo::NIB ? 0 : 2 * 16 * PNS;  // float4 per set
       float4* NI = reinterpret_cast<float4*>(smem + Lo::scratch);
-      float4* NS = NI + 2 * 16 * PNI;
-      if constexpr (PNI > 0) {
-        constexpr int CPN = 4 / Lo::MI;  // coordinates per nibble
-        for (int i = threadIdx.x; i < 2 * 16 * PNI; i += kThreads) {
-          const int pp = i % PNI, n = (i / PNI) % 16, hf = i / (16 * PNI);
-          float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+      float4* NS = NI + NSET * NIS;
 #pragma unroll
-          for (int f = 0; f < CPN; ++f) {
-            const float4 x = *reinterpret_cast<const float4*>(qrT + (2 * CPN * pp + CPN * hf + f) * kMaxHeads);
-            const float c = cenI[(n >> (Lo::MI * f)) & ((1 << Lo::MI) - 1)] * cI;
-            r.x = fmaf(x.x, c, r.x); r.y = fmaf(x.y, c, r.y);
-            r.z = fmaf(x.z, c, r.z); r.w = fmaf(x.w, c, r.w);
+      for (int st = 0; st < NSET; ++st) {
+        if constexpr (PNI > 0) {
+          constexpr int CPN = 4 / Lo::MI;  // coordinates per nibble
+          for (int i = threadIdx.x; i < NIS; i += NT) {
+            const int pp = i % PNI, n = (i / PNI) % 16, hf = i / (16 * PNI);
+            float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int f = 0; f < CPN; ++f) {
+              const float4 x = *reinterpret_cast<const float4*>(qrT + (2 * CPN * pp + CPN * hf + f) * SL + 4 * st);
+              const float c = cenI[(n >> (Lo::MI * f)) & ((1 << Lo::MI) - 1)] * cI;
+              r.x = fmaf(x.x, c, r.x); r.y = fmaf(x.y, c, r.y);
+              r.z = fmaf(x.z, c, r.z); r.w = fmaf(x.w, c, r.w);
+            }
+            NI[st * NIS + (hf * 16 + n) * PNI + pp] = r;
           }
-          NI[(hf * 16 + n) * PNI + pp] = r;
         }
-      }
-      if constexpr (PNS > 0) {
-        for (int i = threadIdx.x; i < 2 * 16 * PNS; i += kThreads) {
-          const int pp = i % PNS, n = (i / PNS) % 16, hf = i / (16 * PNS);
-          float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-          if constexpr (PROD) {
+        if constexpr (Lo::NIB) {
+          // two sets: QJL sign nibble tables built directly, entry n of nibble position np =
+          // sum_f (bit f of n ? +1 : -1) cS Sq_{4 np + f}
+          for (int i = threadIdx.x; i < 16 * 32; i += NT) {
+            const int np = i % 32, n = i / 32;
+            float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int f = 0; f < 4; ++f) {
-              const float4 x = *reinterpret_cast<const float4*>(sqT + (8 * pp + 4 * hf + f) * kMaxHeads);
+              const float4 x = *reinterpret_cast<const float4*>(sqT + (4 * np + f) * SL + 4 * st);
               const float sg = ((n >> f) & 1) ? cS : -cS;
               r.x = fmaf(x.x, sg, r.x); r.y = fmaf(x.y, sg, r.y);
               r.z = fmaf(x.z, sg, r.z); r.w = fmaf(x.w, sg, r.w);
             }
-          } else if (pp < Lo::IBS) {  // grouped normal group; padding positions stay zero
-            constexpr int CPN = 4 / Lo::MS;
-#pragma unroll
-            for (int f = 0; f < CPN; ++f) {
-              const float4 x = *reinterpret_cast<const float4*>(qrT + (32 + 2 * CPN * pp + CPN * hf + f) * kMaxHeads);
-              const float c = cenS[(n >> (Lo::MS * f)) & ((1 << Lo::MS) - 1)] * cS;
-              r.x = fmaf(x.x, c, r.x); r.y = fmaf(x.y, c, r.y);
-              r.z = fmaf(x.z, c, r.z); r.w = fmaf(x.w, c, r.w);
-            }
+            *reinterpret_cast<float4*>(lutS + st * Lo::SETS + (n * 32 + np) * 16) = r;
           }
-          NS[(hf * 16 + n) * PNS + pp] = r;
+        } else if constexpr (PNS > 0) {
+          for (int i = threadIdx.x; i < NSS; i += NT) {
+            const int pp = i % PNS, n = (i / PNS) % 16, hf = i / (16 * PNS);
+            float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+            if constexpr (PROD) {
+#pragma unroll
+              for (int f = 0; f < 4; ++f) {
+                const float4 x = *reinterpret_cast<const float4*>(sqT + (8 * pp + 4 * hf + f) * SL + 4 * st);
+                const float sg = ((n >> f) & 1) ? cS : -cS;
+                r.x = fmaf(x.x, sg, r.x); r.y = fmaf(x.y, sg, r.y);
+                r.z = fmaf(x.z, sg, r.z); r.w = fmaf(x.w, sg, r.w);
+              }
+            } else if (pp < Lo::IBS) {  // grouped normal group; padding positions stay zero
+              constexpr int CPN = 4 / Lo::MS;
+#pragma unroll
+              for (int f = 0; f < CPN; ++f) {
+                const float4 x = *reinterpret_cast<const float4*>(qrT + (32 + 2 * CPN * pp + CPN * hf + f) * SL + 4 * st);
+                const float c = cenS[(n >> (Lo::MS * f)) & ((1 << Lo::MS) - 1)] * cS;
+                r.x = fmaf(x.x, c, r.x); r.y = fmaf(x.y, c, r.y);
+                r.z = fmaf(x.z, c, r.z); r.w = fmaf(x.w, c, r.w);
+              }
+            }
+            NS[st * NSS + (hf * 16 + n) * PNS + pp] = r;
+          }
         }
       }
       __syncthreads();
       // bytes of two 3-bit codes in nibbles: coordinates c0 + 2p, c0 + 2p + 1 (entry e: codes
       // e mod 8 and e / 8)
-      auto build3 = [&](uint8_t* lut, int P, int c0, const float* cen, float cs) {
-        for (int i = threadIdx.x; i < 32 * P; i += kThreads) {
+      auto build3 = [&](uint8_t* lut, int P, int c0, const float* cen, float cs, int st) {
+        for (int i = threadIdx.x; i < 32 * P; i += NT) {
           const int p = i % P, e = i / P;
-          const float4 x = *reinterpret_cast<const float4*>(qrT + (c0 + 2 * p) * kMaxHeads);
-          const float4 y = *reinterpret_cast<const float4*>(qrT + (c0 + 2 * p + 1) * kMaxHeads);
+          const float4 x = *reinterpret_cast<const float4*>(qrT + (c0 + 2 * p) * SL + 4 * st);
+          const float4 y = *reinterpret_cast<const float4*>(qrT + (c0 + 2 * p + 1) * SL + 4 * st);
           const float ca = cen[e & 7] * cs, cb = cen[e >> 3] * cs;
           *reinterpret_cast<float4*>(lut + (e * P + p) * 16) =
               make_float4(fmaf(x.x, ca, y.x * cb), fmaf(x.y, ca, y.y * cb),
@@ -503,22 +580,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         }
       };
       auto compose = [&](uint8_t* lut, const float4* N, int P) {
-        for (int i = threadIdx.x; i < 128 * P; i += kThreads) {
+        for (int i = threadIdx.x; i < 128 * P; i += NT) {
           const int pp = i % P, e = i / P;
           const float4 u = N[(e & 15) * P + pp], v = N[(16 + (e >> 4)) * P + pp];
           *reinterpret_cast<float4*>(lut + (e * P + pp) * 16) =
               make_float4(u.x + v.x, u.y + v.y, u.z + v.z, u.w + v.w);
         }
       };
-      if constexpr (Lo::MI == 3) build3(lutI, PI, 0, cenI, cI);
-      else compose(lutI, NI, PI);
-      if constexpr (GRP && Lo::MS == 3) build3(lutS, PS, 32, cenS, cS);
-      else if constexpr (PS > 0) compose(lutS, NS, PS);
+#pragma unroll
+      for (int st = 0; st < NSET; ++st) {
+        if constexpr (Lo::MI == 3) build3(lutI + st * Lo::SETI, PI, 0, cenI, cI, st);
+        else compose(lutI + st * Lo::SETI, NI + st * NIS, PI);
+        if constexpr (GRP && Lo::MS == 3) build3(lutS + st * Lo::SETS, PS, 32, cenS, cS, st);
+        else if constexpr (PS > 0 && !Lo::NIB) compose(lutS + st * Lo::SETS, NS + st * NSS, PS);
+      }
     }
     __syncthreads();
 
     // ---------------- main loop: this warp's chunks
-    ulonglong2* sPP = reinterpret_cast<ulonglong2*>(smem + Lo::ppair) + warp * 2 * 32;
+    // p pairs of the chunk's tokens: sPP[k 32 + token] = ((p_2k, p_2k), (p_2k+1, p_2k+1))
+    ulonglong2* sPP = reinterpret_cast<ulonglong2*>(smem + Lo::ppair) + warp * (SL / 2) * 32;
     float4* sVP = reinterpret_cast<float4*>(smem + Lo::vpair) + warp * 4 * kVpStride;
     const uint32_t r8 = static_cast<uint32_t>(lane & 7);
     const bool swap = r8 >= 4;
@@ -527,23 +608,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
 #pragma unroll
     for (int i = 0; i < 8; ++i) rot16[i] = ((r8 + i) & 7) * 16;
 
-    for (int ts = c0; ts < t1; ts += kChunkStride) {
+    for (int ts = c0; ts < t1; ts += CS) {
       // prefetch the next chunk's key bytes
       uint32_t nkw[KW], nsw[4], nnw;
-      const int tn = ts + kChunkStride;
+      const int tn = ts + CS;
       if (tn < t1) load_keys(tn, nkw, nsw, nnw);
       const int wcount = min(32, t1 - ts);
       const bool valid = lane < wcount;
 
-      uint64_t accI[2] = {0ull, 0ull}, accS[2] = {0ull, 0ull};
-      if constexpr (PROD) segment_lookups<1, 16>(accS, sw4, lutS, swap, sh, rot16);
-      if constexpr (GRP) segment_lookups<Lo::MS, Lo::PS>(accS, kw + Lo::IBI / 4, lutS, swap, sh, rot16);
-      segment_lookups<Lo::MI, PI>(accI, kw, lutI, swap, sh, rot16);
-      const float n16 = half_lo(nw), r16 = TWO ? half_hi(nw) : 0.f;
-      float sc[kMaxHeads];
+      uint64_t accI[NSET][2], accS[NSET][2];
 #pragma unroll
-      for (int j = 0; j < kMaxHeads / 2; ++j) {
-        const float2 xi = up2(accI[j]), xs = up2(accS[j]);
+      for (int st = 0; st < NSET; ++st) accI[st][0] = accI[st][1] = accS[st][0] = accS[st][1] = 0ull;
+      if constexpr (Lo::NIB) nibble_lookups<NSET, Lo::SETS>(accS, sw4, lutS, r8, rot16);
+      else if constexpr (PROD) segment_lookups<1, 16, NSET, Lo::SETS>(accS, sw4, lutS, swap, sh, rot16);
+      if constexpr (GRP)
+        segment_lookups<Lo::MS, Lo::PS, NSET, Lo::SETS>(accS, kw + Lo::IBI / 4, lutS, swap, sh, rot16);
+      segment_lookups<Lo::MI, PI, NSET, Lo::SETI>(accI, kw, lutI, swap, sh, rot16);
+      const float n16 = half_lo(nw), r16 = TWO ? half_hi(nw) : 0.f;
+      float sc[SL];
+#pragma unroll
+      for (int j = 0; j < SL / 2; ++j) {
+        const float2 xi = up2(accI[j / 2][j % 2]), xs = up2(accS[j / 2][j % 2]);
         sc[2 * j] = TWO ? fmaf(n16, xi.x, r16 * xs.x) : n16 * xi.x;
         sc[2 * j + 1] = TWO ? fmaf(n16, xi.y, r16 * xs.y) : n16 * xi.y;
       }
@@ -570,15 +655,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
           l[h] = fmaf(l[h], alpha, p[h]);
           const uint64_t al = pk2(alpha, alpha);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) o[h][k] = mul2(o[h][k], al);
+          for (int k = 0; k < OC; ++k) o[h][k] = mul2(o[h][k], al);
           m[h] = mn;
         }
         {
-          float pp[kMaxHeads];  // p of the head slots, zero past NH
+          float pp[SL];  // p of the head slots, zero past NH
 #pragma unroll
-          for (int h = 0; h < kMaxHeads; ++h) pp[h] = h < NH ? p[h < NH ? h : 0] : 0.f;
-          sPP[lane] = make_ulonglong2(pk2(pp[0], pp[0]), pk2(pp[1], pp[1]));
-          if constexpr (NH > 2) sPP[32 + lane] = make_ulonglong2(pk2(pp[2], pp[2]), pk2(pp[3], pp[3]));
+          for (int h = 0; h < SL; ++h) pp[h] = h < NH ? p[h < NH ? h : 0] : 0.f;
+#pragma unroll
+          for (int k = 0; k < (NH + 1) / 2; ++k)
+            sPP[k * 32 + lane] = make_ulonglong2(pk2(pp[2 * k], pp[2 * k]), pk2(pp[2 * k + 1], pp[2 * k + 1]));
         }
         cp_async_wait<0>();
         __syncwarp();
@@ -595,41 +681,75 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         }
         __syncwarp();
 
-        // P.V: token 2 jj + hw of the chunk per step, 8 channels per lane (group j16 / 4)
-        const int hw = lane >> 4, j16 = lane & 15, vg = j16 >> 2;
+        if constexpr (NSET == 1) {
+          // P.V: token 2 jj + hw of the chunk per step, 8 channels per lane (group j16 / 4)
+          const int hw = lane >> 4, j16 = lane & 15, vg = j16 >> 2;
+  #pragma unroll 2
+          for (int jj = 0; 2 * jj < wcount; ++jj) {
+            const int tok = 2 * jj + hw;
+            if (tok < wcount) {
+              const float4 dq = sVP[vg * kVpStride + tok];
+              const uint64_t S16 = pk2(dq.x, dq.y), CC = pk2(dq.z, dq.w);
+              uint32_t cw[8];
+              if constexpr (VB == 2) {
+                const uint32_t c16 = reinterpret_cast<const uint16_t*>(wslot + Lo::o_vq + tok * 32)[j16];
+  #pragma unroll
+                for (int k = 0; k < 8; ++k) cw[k] = (c16 << (19 - 2 * k)) & 0x00180000u;
+              } else {
+                const uint32_t c32 = reinterpret_cast<const uint32_t*>(wslot + Lo::o_vq + tok * 64)[j16];
+  #pragma unroll
+                for (int k = 0; k < 8; ++k)
+                  cw[k] = (k < 5 ? (c32 << (19 - 4 * k)) : (c32 >> (4 * k - 19))) & 0x00780000u;
+              }
+              uint64_t v[4];
+  #pragma unroll
+              for (int k = 0; k < 4; ++k)
+                v[k] = fma2(pk2(__uint_as_float(0x3f800000u | cw[2 * k]), __uint_as_float(0x3f800000u | cw[2 * k + 1])), S16, CC);
+              const ulonglong2 p01 = sPP[tok];
+  #pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                o[0][k] = fma2(p01.x, v[k], o[0][k]);
+                if constexpr (NH > 1) o[1][k] = fma2(p01.y, v[k], o[1][k]);
+              }
+              if constexpr (NH > 2) {
+                const ulonglong2 p23 = sPP[32 + tok];
+  #pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  o[2][k] = fma2(p23.x, v[k], o[2][k]);
+                  if constexpr (NH > 3) o[3][k] = fma2(p23.y, v[k], o[3][k]);
+                }
+              }
+            }
+          }
+        } else {
+          // P.V: one token of the chunk per step, channels 4 lane .. 4 lane + 3 (group lane / 8)
+          const int vg = lane >> 3;
 #pragma unroll 2
-        for (int jj = 0; 2 * jj < wcount; ++jj) {
-          const int tok = 2 * jj + hw;
-          if (tok < wcount) {
+          for (int tok = 0; tok < wcount; ++tok) {
             const float4 dq = sVP[vg * kVpStride + tok];
             const uint64_t S16 = pk2(dq.x, dq.y), CC = pk2(dq.z, dq.w);
-            uint32_t cw[8];
+            uint32_t cw[4];
             if constexpr (VB == 2) {
-              const uint32_t c16 = reinterpret_cast<const uint16_t*>(wslot + Lo::o_vq + tok * 32)[j16];
+              const uint32_t c8 = wslot[Lo::o_vq + tok * 32 + lane];
 #pragma unroll
-              for (int k = 0; k < 8; ++k) cw[k] = (c16 << (19 - 2 * k)) & 0x00180000u;
+              for (int k = 0; k < 4; ++k) cw[k] = (c8 << (19 - 2 * k)) & 0x00180000u;
             } else {
-              const uint32_t c32 = reinterpret_cast<const uint32_t*>(wslot + Lo::o_vq + tok * 64)[j16];
+              const uint32_t c16 = reinterpret_cast<const uint16_t*>(wslot + Lo::o_vq + tok * 64)[lane];
 #pragma unroll
-              for (int k = 0; k < 8; ++k)
-                cw[k] = (k < 5 ? (c32 << (19 - 4 * k)) : (c32 >> (4 * k - 19))) & 0x00780000u;
+              for (int k = 0; k < 4; ++k) cw[k] = (c16 << (19 - 4 * k)) & 0x00780000u;
             }
-            uint64_t v[4];
+            uint64_t v[2];
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
+            for (int k = 0; k < 2; ++k)
               v[k] = fma2(pk2(__uint_as_float(0x3f800000u | cw[2 * k]), __uint_as_float(0x3f800000u | cw[2 * k + 1])), S16, CC);
-            const ulonglong2 p01 = sPP[tok];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              o[0][k] = fma2(p01.x, v[k], o[0][k]);
-              if constexpr (NH > 1) o[1][k] = fma2(p01.y, v[k], o[1][k]);
-            }
-            if constexpr (NH > 2) {
-              const ulonglong2 p23 = sPP[32 + tok];
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                o[2][k] = fma2(p23.x, v[k], o[2][k]);
-                if constexpr (NH > 3) o[3][k] = fma2(p23.y, v[k], o[3][k]);
+            for (int k = 0; k < (NH + 1) / 2; ++k) {
+              const ulonglong2 pq = sPP[k * 32 + tok];
+              o[2 * k][0] = fma2(pq.x, v[0], o[2 * k][0]);
+              o[2 * k][1] = fma2(pq.x, v[1], o[2 * k][1]);
+              if (2 * k + 1 < NH) {
+                o[(2 * k + 1) % NH][0] = fma2(pq.y, v[0], o[(2 * k + 1) % NH][0]);
+                o[(2 * k + 1) % NH][1] = fma2(pq.y, v[1], o[(2 * k + 1) % NH][1]);
               }
             }
           }
@@ -654,20 +774,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
   float* sM = reinterpret_cast<float*>(smem + Lo::wv);  // [warp][head][kPartStride]
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
-    // the two half-warps hold disjoint tokens of the same channels
+    if constexpr (NSET == 1) {
+      // the two half-warps hold disjoint tokens of the same channels
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 v = up2(o[h][k]);
-      o[h][k] = add2(o[h][k], pk2(__shfl_xor_sync(kFull, v.x, 16), __shfl_xor_sync(kFull, v.y, 16)));
+      for (int k = 0; k < OC; ++k) {
+        const float2 v = up2(o[h][k]);
+        o[h][k] = add2(o[h][k], pk2(__shfl_xor_sync(kFull, v.x, 16), __shfl_xor_sync(kFull, v.y, 16)));
+      }
     }
     if (h < nh) {
       const float lt = warp_sum(l[h]);
-      float* dst = sM + (warp * kMaxHeads + h) * kPartStride;
+      float* dst = sM + (warp * SL + h) * kPartStride;
       if (lane == 0) { dst[0] = m[h]; dst[1] = lt; }
-      if (lane < 16) {
-        const float2 v0 = up2(o[h][0]), v1 = up2(o[h][1]), v2 = up2(o[h][2]), v3 = up2(o[h][3]);
-        *reinterpret_cast<float4*>(dst + 4 + 8 * lane) = make_float4(v0.x, v0.y, v1.x, v1.y);
-        *reinterpret_cast<float4*>(dst + 8 + 8 * lane) = make_float4(v2.x, v2.y, v3.x, v3.y);
+      if constexpr (NSET == 1) {
+        if (lane < 16) {
+          const float2 v0 = up2(o[h][0]), v1 = up2(o[h][1]), v2 = up2(o[h][2 % OC]), v3 = up2(o[h][3 % OC]);
+          *reinterpret_cast<float4*>(dst + 4 + 8 * lane) = make_float4(v0.x, v0.y, v1.x, v1.y);
+          *reinterpret_cast<float4*>(dst + 8 + 8 * lane) = make_float4(v2.x, v2.y, v3.x, v3.y);
+        }
+      } else {
+        const float2 v0 = up2(o[h][0]), v1 = up2(o[h][1]);
+        *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = make_float4(v0.x, v0.y, v1.x, v1.y);
       }
     }
   }
@@ -676,12 +803,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
     const int h = warp, hq = a.g_heads[grp][h];
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sM[(w * kMaxHeads + h) * kPartStride]);
+    for (int w = 0; w < NWp; ++w) M = fmaxf(M, sM[(w * SL + h) * kPartStride]);
     float Lsum = 0.f, O[4] = {0.f, 0.f, 0.f, 0.f};
     if (M != -INFINITY) {
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const float* src = sM + (w * kMaxHeads + h) * kPartStride;
+      for (int w = 0; w < NWp; ++w) {
+        const float* src = sM + (w * SL + h) * kPartStride;
         if (src[0] == -INFINITY) continue;
         const float f = exp2f(src[0] - M);
         Lsum = fmaf(f, src[1], Lsum);
@@ -734,12 +861,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
   {
     const int S = a.n_splits;
     float* sMx = reinterpret_cast<float*>(smem + Lo::wv);   // [head][S] split maxima
-    float* sLs = sMx + kMaxHeads * 256;                      // [head][S] split sums
-    float* sF = sLs + kMaxHeads * 256;                       // [head][S] weights
-    float* sHd = sF + kMaxHeads * 256;  // [head] 1 / total sum, then [head] maxima and sums
-    float4* sAcc = reinterpret_cast<float4*>(sHd + 16);      // [slice][head][32]
+    float* sLs = sMx + SL * 256;                      // [head][S] split sums
+    float* sF = sLs + SL * 256;                       // [head][S] weights
+    float* sHd = sF + SL * 256;  // [head] 1 / total sum, then [head] maxima and sums
+    float4* sAcc = reinterpret_cast<float4*>(sHd + 4 * SL);      // [slice][head][32]
     const float* base = a.part + static_cast<int64_t>(b) * a.n_q_heads * S * kPartStride;
-    for (int i = threadIdx.x; i < nh * S; i += kThreads) {
+    for (int i = threadIdx.x; i < nh * S; i += NT) {
       const int h = i / S, sp = i - h * S;
       const float* src = base + (static_cast<int64_t>(a.g_heads[grp][h]) * S + sp) * kPartStride;
       sMx[h * 256 + sp] = __ldcg(src);
@@ -761,12 +888,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
       lsum = warp_sum(lsum);
       if (lane == 0) {
         sHd[h] = lsum > 0.f ? 1.f / lsum : 0.f;
-        sHd[kMaxHeads + h] = M;
-        sHd[2 * kMaxHeads + h] = lsum;
+        sHd[SL + h] = M;
+        sHd[2 * SL + h] = lsum;
       }
     }
     __syncthreads();
-    const int G = kThreads / (32 * nh);  // split slices
+    const int G = NT / (32 * nh);  // split slices
     if (threadIdx.x < G * 32 * nh) {
       const int h = threadIdx.x / (32 * G), r = threadIdx.x - h * 32 * G;
       const int qd = r & 31, g = r >> 5;
@@ -790,21 +917,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
         acc.x = fmaf(f, v.x, acc.x); acc.y = fmaf(f, v.y, acc.y);
         acc.z = fmaf(f, v.z, acc.z); acc.w = fmaf(f, v.w, acc.w);
       }
-      sAcc[(g * kMaxHeads + h) * 32 + qd] = acc;
+      sAcc[(g * nh + h) * 32 + qd] = acc;
     }
     __syncthreads();
     if (threadIdx.x < 32 * nh) {
       const int h = threadIdx.x >> 5, qd = threadIdx.x & 31, hq = a.g_heads[grp][h];
       float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int g = 0; g < G; ++g) {
-        const float4 v = sAcc[(g * kMaxHeads + h) * 32 + qd];
+        const float4 v = sAcc[(g * nh + h) * 32 + qd];
         O.x += v.x; O.y += v.y; O.z += v.z; O.w += v.w;
       }
       const float inv = sHd[h];
       const int64_t orow = (static_cast<int64_t>(b) * a.n_q_heads + hq) * kD + 4 * qd;
       if (a.part_out != nullptr) {
         float* dst = a.part_out + (static_cast<int64_t>(b) * a.n_q_heads + hq) * kPartStride;
-        if (qd == 0) *reinterpret_cast<float4*>(dst) = make_float4(sHd[kMaxHeads + h], sHd[2 * kMaxHeads + h], 0.f, 0.f);
+        if (qd == 0) *reinterpret_cast<float4*>(dst) = make_float4(sHd[SL + h], sHd[2 * SL + h], 0.f, 0.f);
         *reinterpret_cast<float4*>(dst + 4 + 4 * qd) = O;
       } else if (a.out_f32) {
         *reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow) =
@@ -822,10 +949,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode(const __grid_constant__ 
   if (threadIdx.x == 0) a.counters[static_cast<int64_t>(b) * a.n_q_heads + a.g_heads[grp][0]] = 0;
 }
 
-template <int MB, int VB, int NH, int K>
+template <int MB, int VB, int NH, int K, int NSET>
 tq_status run_decode(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
-  constexpr int smem = Lay<MB, VB, K>::total;
-  auto kern = k_decode<MB, VB, NH, K>;
+  constexpr int smem = Lay<MB, VB, K, NSET>::total;
+  auto kern = k_decode<MB, VB, NH, K, NSET>;
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
@@ -835,7 +962,7 @@ tq_status run_decode(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(Cfg<NSET>::threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -849,9 +976,9 @@ tq_status run_decode(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
 
 template <int MB, int VB, int K>
 tq_status run_decode_nh(const DecodeArgs& a, dim3 grid, int max_heads, cudaStream_t st) {
-  if (max_heads <= 2) return run_decode<MB, VB, 2, K>(a, grid, st);
-  if (max_heads == 3) return run_decode<MB, VB, 3, K>(a, grid, st);
-  return run_decode<MB, VB, 4, K>(a, grid, st);
+  if (max_heads <= 2) return run_decode<MB, VB, 2, K, 1>(a, grid, st);
+  if (max_heads == 3) return run_decode<MB, VB, 3, K, 1>(a, grid, st);
+  return run_decode<MB, VB, 4, K, 1>(a, grid, st);
 }
 
 // LSE merge of context-split partial records (m, l, o) of n_parts slices: per row (sequence,
@@ -890,6 +1017,62 @@ __global__ void __launch_bounds__(128) k_merge_partials(const float* __restrict_
     pk.x = *reinterpret_cast<uint32_t*>(&lo);
     pk.y = *reinterpret_cast<uint32_t*>(&hi);
     *reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + orow) = pk;
+  }
+}
+
+// Two table sets (up to 8 heads per CTA, 12 warps) where the layout fits; grouped keys and
+// configurations whose two-set tables exceed the shared memory keep one set.
+template <int MB, int VB, int K>
+constexpr bool two_sets_fit() {
+  if constexpr (K == kGrp) return false;
+  else return Lay<MB, VB, K, 2>::fits;
+}
+
+template <int MB, int VB, int K>
+tq_status run_decode_sets(const DecodeArgs& a, dim3 grid, int max_heads, bool two,
+                          cudaStream_t st) {
+  if constexpr (two_sets_fit<MB, VB, K>()) {
+    if (two) {
+      if (max_heads <= 6) return run_decode<MB, VB, 6, K, 2>(a, grid, st);
+      return run_decode<MB, VB, 8, K, 2>(a, grid, st);
+    }
+  }
+  return run_decode_nh<MB, VB, K>(a, grid, max_heads, st);
+}
+
+bool two_sets_ok(int kind, int mb, int vb) {
+  switch (kind * 64 + mb * 8 + vb) {
+    case kProd * 64 + 1 * 8 + 0: return two_sets_fit<1, 0, kProd>();
+    case kProd * 64 + 1 * 8 + 2: return two_sets_fit<1, 2, kProd>();
+    case kProd * 64 + 1 * 8 + 4: return two_sets_fit<1, 4, kProd>();
+    case kProd * 64 + 2 * 8 + 0: return two_sets_fit<2, 0, kProd>();
+    case kProd * 64 + 2 * 8 + 2: return two_sets_fit<2, 2, kProd>();
+    case kProd * 64 + 2 * 8 + 4: return two_sets_fit<2, 4, kProd>();
+    case kProd * 64 + 3 * 8 + 0: return two_sets_fit<3, 0, kProd>();
+    case kProd * 64 + 3 * 8 + 2: return two_sets_fit<3, 2, kProd>();
+    case kProd * 64 + 3 * 8 + 4: return two_sets_fit<3, 4, kProd>();
+    case kMse * 64 + 1 * 8 + 0: return two_sets_fit<1, 0, kMse>();
+    case kMse * 64 + 1 * 8 + 2: return two_sets_fit<1, 2, kMse>();
+    case kMse * 64 + 1 * 8 + 4: return two_sets_fit<1, 4, kMse>();
+    case kMse * 64 + 2 * 8 + 0: return two_sets_fit<2, 0, kMse>();
+    case kMse * 64 + 2 * 8 + 2: return two_sets_fit<2, 2, kMse>();
+    case kMse * 64 + 2 * 8 + 4: return two_sets_fit<2, 4, kMse>();
+    case kMse * 64 + 3 * 8 + 0: return two_sets_fit<3, 0, kMse>();
+    case kMse * 64 + 3 * 8 + 2: return two_sets_fit<3, 2, kMse>();
+    case kMse * 64 + 3 * 8 + 4: return two_sets_fit<3, 4, kMse>();
+    case kMse * 64 + 4 * 8 + 0: return two_sets_fit<4, 0, kMse>();
+    case kMse * 64 + 4 * 8 + 2: return two_sets_fit<4, 2, kMse>();
+    case kMse * 64 + 4 * 8 + 4: return two_sets_fit<4, 4, kMse>();
+    case kGrp * 64 + 1 * 8 + 0: return two_sets_fit<1, 0, kGrp>();
+    case kGrp * 64 + 1 * 8 + 2: return two_sets_fit<1, 2, kGrp>();
+    case kGrp * 64 + 1 * 8 + 4: return two_sets_fit<1, 4, kGrp>();
+    case kGrp * 64 + 2 * 8 + 0: return two_sets_fit<2, 0, kGrp>();
+    case kGrp * 64 + 2 * 8 + 2: return two_sets_fit<2, 2, kGrp>();
+    case kGrp * 64 + 2 * 8 + 4: return two_sets_fit<2, 4, kGrp>();
+    case kGrp * 64 + 3 * 8 + 0: return two_sets_fit<3, 0, kGrp>();
+    case kGrp * 64 + 3 * 8 + 2: return two_sets_fit<3, 2, kGrp>();
+    case kGrp * 64 + 3 * 8 + 4: return two_sets_fit<3, 4, kGrp>();
+    default: return false;
   }
 }
 
@@ -942,7 +1125,38 @@ tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* c, const void*
   a.scale_log2 = scale * 1.4426950408889634074f;
   a.inv_scale_log2 = 1.f / a.scale_log2;
 
-  // head groups: the query heads of each KV head, in balanced groups of at most 4
+  // key kind and widths (MB: index bits, prod: bits - 1; grouped: the base bits)
+  const int kind = q->mode == TQ_MODE_PROD ? kProd : (q->mode == TQ_MODE_GROUPED ? kGrp : kMse);
+  const int mb = kind == kProd ? q->bits - 1 : q->bits;
+  const int vb = c->value_bits;
+
+  int max_len = 0;
+  for (int b = 0; b < c->batch; ++b) max_len = c->len_host[b] > max_len ? c->len_host[b] : max_len;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int sms = std::max(1, sm_count(dev) - 4);
+
+  // The query heads of each KV head; a CTA serves up to 8 of them (two table sets) where some
+  // KV head has more than 4, the two-set layout fits, and the decode is large enough to
+  // amortise the two-set CTA's longer fixed path (its prologue builds twice the tables and
+  // its chunks carry twice the heads): at least 4 chunk rounds of (token, KV head) units per
+  // SM. Measured: 1.05 M units (batch 8 x 4 KV heads x 32768, or 1 x 8 x 131072) run 11-16 %
+  // faster with two sets; 65536 units (1 x 2 x 32768) run 16 % slower. tq_set_decode_policy
+  // can force either shape.
+  int per_kv_max = 0;
+  for (int kv = 0; kv < c->n_kv_heads; ++kv) {
+    int n = 0;
+    for (int h = 0; h < n_q_heads; ++h)
+      if ((head_map ? head_map[h] : h / (n_q_heads / c->n_kv_heads)) == kv) ++n;
+    per_kv_max = n > per_kv_max ? n : per_kv_max;
+  }
+  const long long units = static_cast<long long>(c->batch) * c->n_kv_heads * max_len;
+  const int policy = g_decode_policy.load(std::memory_order_relaxed);
+  const bool two = per_kv_max > kMaxHeads && two_sets_ok(kind, mb, vb) &&
+                   policy != TQ_DECODE_ONE_SET &&
+                   (policy == TQ_DECODE_TWO_SETS || units >= 4ll * Cfg<2>::chunk_stride * sms);
+  const int cap = two ? kMaxSlots : kMaxHeads;
+  // head groups: the query heads of each KV head, in balanced groups of at most `cap`
   int n_groups = 0, max_heads = 0;
   for (int kv = 0; kv < c->n_kv_heads; ++kv) {
     int heads[1024];
@@ -950,7 +1164,7 @@ tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* c, const void*
     for (int h = 0; h < n_q_heads; ++h)
       if ((head_map ? head_map[h] : h / (n_q_heads / c->n_kv_heads)) == kv) heads[n++] = h;
     if (n == 0) continue;
-    const int ng = (n + kMaxHeads - 1) / kMaxHeads;
+    const int ng = (n + cap - 1) / cap;
     int pos = 0;
     for (int g = 0; g < ng; ++g) {
       const int cnt = (n - pos) / (ng - g);
@@ -965,17 +1179,12 @@ tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* c, const void*
   }
   if (n_groups == 0) return TQ_OK;
 
-  int max_len = 0;
-  for (int b = 0; b < c->batch; ++b) max_len = c->len_host[b] > max_len ? c->len_host[b] : max_len;
   if (max_len == 0 && out == nullptr && part_out == nullptr) return TQ_OK;
 
   // split count: one CTA per SM; minimise waves x (tokens per split + per-CTA set-up) + the
   // final combine (its loads grow with the number of splits). A few SMs are left out of the
   // first wave so that an append kernel still resident on them does not hold back a CTA of
   // this grid when it starts early (programmatic dependent launch).
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const int sms = std::max(1, sm_count(dev) - 4);
   const int pairs = c->batch * n_groups;
   const int cap_splits = max_splits_for(c->capacity);
   int best = 1;
@@ -986,7 +1195,8 @@ tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* c, const void*
     const int used = (max_len + tps - 1) / tps;
     if (used != s) continue;
     const double waves = std::ceil(static_cast<double>(pairs) * s / sms);
-    const double cost = waves * (tps + 512.0) + (s > 1 ? 8.0 * s : 0.0);
+    const double cost = waves * (tps + (two ? Cfg<2>::chunk_stride : Cfg<1>::chunk_stride)) +
+                        (s > 1 ? 8.0 * s : 0.0);
     if (cost < best_cost - 1e-9) { best_cost = cost; best = s; }
   }
   a.n_splits = best;
@@ -998,41 +1208,37 @@ tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* c, const void*
   a.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + ((parts + 255) / 256) * 256);
 
   const dim3 grid(a.n_splits, n_groups, c->batch);
-  // MB: index bits (prod: bits - 1) or the grouped base bits
-  const int kind = q->mode == TQ_MODE_PROD ? kProd : (q->mode == TQ_MODE_GROUPED ? kGrp : kMse);
-  const int mb = kind == kProd ? q->bits - 1 : q->bits;
-  const int vb = c->value_bits;
   switch (kind * 64 + mb * 8 + vb) {
-    case kProd * 64 + 1 * 8 + 0: return run_decode_nh<1, 0, kProd>(a, grid, max_heads, st);
-    case kProd * 64 + 1 * 8 + 2: return run_decode_nh<1, 2, kProd>(a, grid, max_heads, st);
-    case kProd * 64 + 1 * 8 + 4: return run_decode_nh<1, 4, kProd>(a, grid, max_heads, st);
-    case kProd * 64 + 2 * 8 + 0: return run_decode_nh<2, 0, kProd>(a, grid, max_heads, st);
-    case kProd * 64 + 2 * 8 + 2: return run_decode_nh<2, 2, kProd>(a, grid, max_heads, st);
-    case kProd * 64 + 2 * 8 + 4: return run_decode_nh<2, 4, kProd>(a, grid, max_heads, st);
-    case kProd * 64 + 3 * 8 + 0: return run_decode_nh<3, 0, kProd>(a, grid, max_heads, st);
-    case kProd * 64 + 3 * 8 + 2: return run_decode_nh<3, 2, kProd>(a, grid, max_heads, st);
-    case kProd * 64 + 3 * 8 + 4: return run_decode_nh<3, 4, kProd>(a, grid, max_heads, st);
-    case kMse * 64 + 1 * 8 + 0: return run_decode_nh<1, 0, kMse>(a, grid, max_heads, st);
-    case kMse * 64 + 1 * 8 + 2: return run_decode_nh<1, 2, kMse>(a, grid, max_heads, st);
-    case kMse * 64 + 1 * 8 + 4: return run_decode_nh<1, 4, kMse>(a, grid, max_heads, st);
-    case kMse * 64 + 2 * 8 + 0: return run_decode_nh<2, 0, kMse>(a, grid, max_heads, st);
-    case kMse * 64 + 2 * 8 + 2: return run_decode_nh<2, 2, kMse>(a, grid, max_heads, st);
-    case kMse * 64 + 2 * 8 + 4: return run_decode_nh<2, 4, kMse>(a, grid, max_heads, st);
-    case kMse * 64 + 3 * 8 + 0: return run_decode_nh<3, 0, kMse>(a, grid, max_heads, st);
-    case kMse * 64 + 3 * 8 + 2: return run_decode_nh<3, 2, kMse>(a, grid, max_heads, st);
-    case kMse * 64 + 3 * 8 + 4: return run_decode_nh<3, 4, kMse>(a, grid, max_heads, st);
-    case kMse * 64 + 4 * 8 + 0: return run_decode_nh<4, 0, kMse>(a, grid, max_heads, st);
-    case kMse * 64 + 4 * 8 + 2: return run_decode_nh<4, 2, kMse>(a, grid, max_heads, st);
-    case kMse * 64 + 4 * 8 + 4: return run_decode_nh<4, 4, kMse>(a, grid, max_heads, st);
-    case kGrp * 64 + 1 * 8 + 0: return run_decode_nh<1, 0, kGrp>(a, grid, max_heads, st);
-    case kGrp * 64 + 1 * 8 + 2: return run_decode_nh<1, 2, kGrp>(a, grid, max_heads, st);
-    case kGrp * 64 + 1 * 8 + 4: return run_decode_nh<1, 4, kGrp>(a, grid, max_heads, st);
-    case kGrp * 64 + 2 * 8 + 0: return run_decode_nh<2, 0, kGrp>(a, grid, max_heads, st);
-    case kGrp * 64 + 2 * 8 + 2: return run_decode_nh<2, 2, kGrp>(a, grid, max_heads, st);
-    case kGrp * 64 + 2 * 8 + 4: return run_decode_nh<2, 4, kGrp>(a, grid, max_heads, st);
-    case kGrp * 64 + 3 * 8 + 0: return run_decode_nh<3, 0, kGrp>(a, grid, max_heads, st);
-    case kGrp * 64 + 3 * 8 + 2: return run_decode_nh<3, 2, kGrp>(a, grid, max_heads, st);
-    case kGrp * 64 + 3 * 8 + 4: return run_decode_nh<3, 4, kGrp>(a, grid, max_heads, st);
+    case kProd * 64 + 1 * 8 + 0: return run_decode_sets<1, 0, kProd>(a, grid, max_heads, two, st);
+    case kProd * 64 + 1 * 8 + 2: return run_decode_sets<1, 2, kProd>(a, grid, max_heads, two, st);
+    case kProd * 64 + 1 * 8 + 4: return run_decode_sets<1, 4, kProd>(a, grid, max_heads, two, st);
+    case kProd * 64 + 2 * 8 + 0: return run_decode_sets<2, 0, kProd>(a, grid, max_heads, two, st);
+    case kProd * 64 + 2 * 8 + 2: return run_decode_sets<2, 2, kProd>(a, grid, max_heads, two, st);
+    case kProd * 64 + 2 * 8 + 4: return run_decode_sets<2, 4, kProd>(a, grid, max_heads, two, st);
+    case kProd * 64 + 3 * 8 + 0: return run_decode_sets<3, 0, kProd>(a, grid, max_heads, two, st);
+    case kProd * 64 + 3 * 8 + 2: return run_decode_sets<3, 2, kProd>(a, grid, max_heads, two, st);
+    case kProd * 64 + 3 * 8 + 4: return run_decode_sets<3, 4, kProd>(a, grid, max_heads, two, st);
+    case kMse * 64 + 1 * 8 + 0: return run_decode_sets<1, 0, kMse>(a, grid, max_heads, two, st);
+    case kMse * 64 + 1 * 8 + 2: return run_decode_sets<1, 2, kMse>(a, grid, max_heads, two, st);
+    case kMse * 64 + 1 * 8 + 4: return run_decode_sets<1, 4, kMse>(a, grid, max_heads, two, st);
+    case kMse * 64 + 2 * 8 + 0: return run_decode_sets<2, 0, kMse>(a, grid, max_heads, two, st);
+    case kMse * 64 + 2 * 8 + 2: return run_decode_sets<2, 2, kMse>(a, grid, max_heads, two, st);
+    case kMse * 64 + 2 * 8 + 4: return run_decode_sets<2, 4, kMse>(a, grid, max_heads, two, st);
+    case kMse * 64 + 3 * 8 + 0: return run_decode_sets<3, 0, kMse>(a, grid, max_heads, two, st);
+    case kMse * 64 + 3 * 8 + 2: return run_decode_sets<3, 2, kMse>(a, grid, max_heads, two, st);
+    case kMse * 64 + 3 * 8 + 4: return run_decode_sets<3, 4, kMse>(a, grid, max_heads, two, st);
+    case kMse * 64 + 4 * 8 + 0: return run_decode_sets<4, 0, kMse>(a, grid, max_heads, two, st);
+    case kMse * 64 + 4 * 8 + 2: return run_decode_sets<4, 2, kMse>(a, grid, max_heads, two, st);
+    case kMse * 64 + 4 * 8 + 4: return run_decode_sets<4, 4, kMse>(a, grid, max_heads, two, st);
+    case kGrp * 64 + 1 * 8 + 0: return run_decode_sets<1, 0, kGrp>(a, grid, max_heads, two, st);
+    case kGrp * 64 + 1 * 8 + 2: return run_decode_sets<1, 2, kGrp>(a, grid, max_heads, two, st);
+    case kGrp * 64 + 1 * 8 + 4: return run_decode_sets<1, 4, kGrp>(a, grid, max_heads, two, st);
+    case kGrp * 64 + 2 * 8 + 0: return run_decode_sets<2, 0, kGrp>(a, grid, max_heads, two, st);
+    case kGrp * 64 + 2 * 8 + 2: return run_decode_sets<2, 2, kGrp>(a, grid, max_heads, two, st);
+    case kGrp * 64 + 2 * 8 + 4: return run_decode_sets<2, 4, kGrp>(a, grid, max_heads, two, st);
+    case kGrp * 64 + 3 * 8 + 0: return run_decode_sets<3, 0, kGrp>(a, grid, max_heads, two, st);
+    case kGrp * 64 + 3 * 8 + 2: return run_decode_sets<3, 2, kGrp>(a, grid, max_heads, two, st);
+    case kGrp * 64 + 3 * 8 + 4: return run_decode_sets<3, 4, kGrp>(a, grid, max_heads, two, st);
     default: return TQ_EUNSUPPORTED;
   }
 }
@@ -1079,6 +1285,14 @@ tq_status launch_decode_noalloc(const tq_quantizer* q, const tq_kv_cache* c, con
     return TQ_ECUDA;
   return launch_decode(q, c, qv, q_dtype, n_q_heads, head_map, sm_scale, out, out_dtype, scores,
                        scores_ld, nullptr, base, need, st);
+}
+
+tq_status set_decode_policy(int policy, int* previous) {
+  if (policy != TQ_DECODE_AUTO && policy != TQ_DECODE_ONE_SET && policy != TQ_DECODE_TWO_SETS)
+    return TQ_EINVAL;
+  const int old = g_decode_policy.exchange(policy);
+  if (previous) *previous = old;
+  return TQ_OK;
 }
 
 }  // namespace tq

@@ -351,6 +351,10 @@ tq_status tq_decode_attention_partial(const tq_quantizer* q, const tq_kv_cache* 
                        0, part, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
+tq_status tq_set_decode_policy(int policy, int* previous) {
+  return set_decode_policy(policy, previous);
+}
+
 tq_status tq_merge_partials(const float* parts, int n_parts, int batch, int n_q_heads, void* out,
                             int out_dtype, void* stream) {
   if (n_parts < 1 || n_parts > 65536 || batch <= 0 || n_q_heads <= 0 || n_q_heads > 512)

@@ -109,6 +109,7 @@ tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* cache, const v
                         int q_dtype, int n_q_heads, const int32_t* head_map, float sm_scale,
                         void* out, int out_dtype, float* scores, int64_t scores_ld,
                         float* part_out, void* workspace, size_t workspace_bytes, cudaStream_t st);
+tq_status set_decode_policy(int policy, int* previous);
 tq_status launch_merge_partials(const float* parts, int n_parts, int64_t rows, void* out,
                                 int out_dtype, cudaStream_t st);
 

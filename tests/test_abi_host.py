@@ -119,3 +119,15 @@ def test_merge_partials_checks_arguments_on_host():
         a = dict(ok, **change)
         assert lib.tq_merge_partials(a["parts"], a["n"], a["b"], a["h"], a["out"], a["dt"],
                                      None) == status, change
+
+
+def test_decode_policy_setter_on_host():
+    prev = tq.tq_set_decode_policy(tq.TQ_DECODE_ONE_SET)
+    try:
+        assert tq.tq_set_decode_policy(tq.TQ_DECODE_TWO_SETS) == tq.TQ_DECODE_ONE_SET
+        with pytest.raises(tq.TQError) as e:
+            tq.tq_set_decode_policy(3)
+        assert e.value.status == tq.TQ_EINVAL
+        assert tq.tq_set_decode_policy(tq.TQ_DECODE_AUTO) == tq.TQ_DECODE_TWO_SETS
+    finally:
+        tq.tq_set_decode_policy(prev)

@@ -318,3 +318,78 @@ def test_decode_context_split_partials_and_merge(mode, bits, vbits):
     tq.tq_merge_partials(whole, out)
     direct, _, _ = run_decode(qg, cache, Q, torch.bfloat16, torch.float32)
     assert np.array_equal(out.cpu().numpy(), direct)
+
+
+@pytest.fixture(params=["two_sets", "one_set"])
+def decode_shape(request):
+    """Force the two-set (up to 8 heads per block) or the one-set decode shape."""
+    pol = tq.TQ_DECODE_TWO_SETS if request.param == "two_sets" else tq.TQ_DECODE_ONE_SET
+    prev = tq.tq_set_decode_policy(pol)
+    yield request.param
+    tq.tq_set_decode_policy(prev)
+
+
+@pytest.fixture
+def two_sets():
+    prev = tq.tq_set_decode_policy(tq.TQ_DECODE_TWO_SETS)
+    yield
+    tq.tq_set_decode_policy(prev)
+
+
+@pytest.mark.parametrize("mode,bits,vbits,hq,hm", [
+    ("prod", 3, 2, 12, None),                                   # 6 heads per KV head
+    ("prod", 3, 2, 14, None),                                   # 7
+    ("prod", 4, 4, 16, None),                                   # 8, 3-bit indices in nibbles
+    ("prod", 2, 4, 10, None),                                   # 5
+    ("mse", 2, 2, 12, None),
+    ("mse", 3, 4, 16, None),
+    ("prod", 3, 2, 11, [0] * 8 + [1] * 3),                      # 8 and 3: one CTA with nh < NH
+])
+def test_decode_eight_heads_per_cta(mode, bits, vbits, hq, hm, decode_shape):
+    """More than 4 query heads per KV head, in both block shapes: one block serving up to 8
+    of them with two table sets (12 warps, nibble sign tables for prod, one token per P.V
+    step), and blocks of at most 4."""
+    require_cuda()
+    qo, qg, oc, cache, Q = small_case(150 + bits + hq, 2, hq, 2, [1000, 613], 1024, bits, vbits, mode)
+    out, sc, _ = run_decode(qg, cache, Q, torch.bfloat16, torch.float32, head_map=hm,
+                            scores_ld=1024)
+    ref, rs = O.decode_attention(qo, oc, Q.astype(np.float64), head_map=hm, value_bits=vbits,
+                                 want_scores=True)
+    err = check_attention(out, ref, False)
+    hmap = hm if hm is not None else O.default_head_map(hq, 2)
+    for b, L in enumerate([1000, 613]):
+        n16 = O.fp16_from_bits(oc["k_norms"][b, :, :L, 0])
+        for h in range(hq):
+            check_scores(sc[b, h, :L], rs[b][h], np.linalg.norm(Q[b, h]), n16[hmap[h]])
+    print(mode, bits, vbits, hq, decode_shape, err)
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_decode_eight_heads_scores_only(bits, two_sets):
+    """Key-only cache (scores, no values) with 8 query heads per KV head."""
+    require_cuda()
+    qo, qg, oc, cache, Q = small_case(170 + bits, 1, 8, 1, [777], 784, bits, 0)
+    _, sc, _ = run_decode(qg, cache, Q, torch.float32, torch.float32, scores_ld=784)
+    _, ref = O.decode_attention(qo, oc, Q.astype(np.float64), value_bits=0, want_scores=True)
+    n16 = O.fp16_from_bits(oc["k_norms"][0, 0, :777, 0])
+    for h in range(8):
+        check_scores(sc[0, h, :777], ref[0][h], np.linalg.norm(Q[0, h]), n16)
+
+
+def test_decode_eight_heads_partials_and_merge(two_sets):
+    """The context-split partial records with two table sets per CTA."""
+    dev = require_cuda()
+    qo, qg, oc, cache, Q = small_case(190, 2, 14, 2, [900, 640], 912, 3, 2)
+    B, Hq = Q.shape[:2]
+    qt = to_device(Q, torch.bfloat16)
+    cuts = (0, 300, 900)
+    parts = torch.empty((2, B, Hq, tq.TQ_PART_FLOATS), device=dev)
+    for i, (a, b) in enumerate(zip(cuts[:-1], cuts[1:])):
+        sl = _slice_oracle_cache(oc, a, b)
+        c = tq.KVCache(qg, B, 2, ((b - a) + 15) // 16 * 16, value_bits=2, device=dev)
+        upload_cache(c, sl)
+        tq.tq_decode_attention_partial(qg, c, qt, parts[i], tq.alloc_decode_workspace(c, Hq))
+    out = torch.empty((B, Hq, 128), device=dev)
+    tq.tq_merge_partials(parts, out)
+    ref, _ = O.decode_attention(qo, oc, Q.astype(np.float64), value_bits=2)
+    check_attention(out.cpu().numpy(), ref, False)
