@@ -104,7 +104,7 @@ struct Cfg {
 // bytes form two lookup segments: I (index bytes; grouped: the outlier group) and S (prod:
 // the QJL sign bytes; grouped: the normal group, padded with zero bytes to whole 8-byte
 // blocks). Each segment accumulates its own sum; the two norms scale them.
-template <int MB, int VB, int K, int NSET>
+template <int MB, int VB, int K, int NSET, bool NIBT = false>
 struct Lay {
   static constexpr int SL = Cfg<NSET>::slots, kWarps = Cfg<NSET>::warps;
   static constexpr bool GRP = K == kGrp;
@@ -121,10 +121,10 @@ struct Lay {
   static constexpr int NB = K == kMse ? 2 : 4;                     // norm bytes per token
   static constexpr int VQB = VB ? kD * VB / 8 : 0;         // value code bytes per token
   static constexpr int VPB = VB ? 16 : 0;                  // value params per token
-  // Tables: NSET sets (head slots 4s .. 4s + 3), each set contiguous. With two sets the
-  // QJL sign tables are nibble tables (16 entries x 32 nibble positions, no mirror), which
-  // keeps two sets of 3-bit prod tables within the shared memory.
-  static constexpr bool NIB = K == kProd && NSET == 2;
+  // Tables: NSET sets (head slots 4s .. 4s + 3), each set contiguous. NIBT: the QJL sign
+  // tables are nibble tables (16 entries x 32 nibble positions, no mirror), which keeps two
+  // sets of 3-bit prod tables within the shared memory.
+  static constexpr bool NIB = NIBT;
   static constexpr int SETI = EI * PI * 16;                          // bytes of one index set
   static constexpr int SETS = NIB ? 16 * 32 * 16 : ES * PS * 16;     // bytes of one sign set
   static constexpr int lutI = 0;
@@ -158,6 +158,14 @@ struct Lay {
   static_assert(IBI % 8 == 0 && PS % 8 == 0, "whole 8-byte lookup blocks");
   static_assert(NSET == 1 || K != kGrp, "grouped keys use one table set");
   static constexpr bool fits = total <= 227 * 1024;                  // decode shared memory budget
+};
+
+// The layout a kernel uses: byte sign tables (16 lookups a key) where they fit, else nibble
+// sign tables (32 lookups a key, 4 times smaller) for two sets of prod tables.
+template <int MB, int VB, int K, int NSET>
+struct LayPick {
+  static constexpr bool nib = K == kProd && NSET == 2 && !Lay<MB, VB, K, NSET, false>::fits;
+  using type = Lay<MB, VB, K, NSET, nib>;
 };
 
 // Accumulate one 4-head table entry of each of the NS table sets (SETB bytes apart) with
@@ -267,7 +275,7 @@ __device__ __forceinline__ void nibble_lookups(uint64_t (&acc)[NS][2], const uin
 // groups (Pi_g: 32-point Hadamard blocks after the group's signs).
 template <int MB, int VB, int NH, int K, int NSET>
 __global__ void __launch_bounds__(Cfg<NSET>::threads, 1) k_decode(const __grid_constant__ DecodeArgs a) {
-  using Lo = Lay<MB, VB, K, NSET>;
+  using Lo = typename LayPick<MB, VB, K, NSET>::type;
   constexpr int NT = Cfg<NSET>::threads, NWp = Cfg<NSET>::warps, CS = Cfg<NSET>::chunk_stride;
   constexpr int SL = Cfg<NSET>::slots;
   constexpr bool PROD = K == kProd, GRP = K == kGrp, TWO = K != kMse;
@@ -951,7 +959,7 @@ __global__ void __launch_bounds__(Cfg<NSET>::threads, 1) k_decode(const __grid_c
 
 template <int MB, int VB, int NH, int K, int NSET>
 tq_status run_decode(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
-  constexpr int smem = Lay<MB, VB, K, NSET>::total;
+  constexpr int smem = LayPick<MB, VB, K, NSET>::type::total;
   auto kern = k_decode<MB, VB, NH, K, NSET>;
   static bool configured = false;
   if (!configured) {
@@ -1025,7 +1033,7 @@ __global__ void __launch_bounds__(128) k_merge_partials(const float* __restrict_
 template <int MB, int VB, int K>
 constexpr bool two_sets_fit() {
   if constexpr (K == kGrp) return false;
-  else return Lay<MB, VB, K, 2>::fits;
+  else return LayPick<MB, VB, K, 2>::type::fits;
 }
 
 template <int MB, int VB, int K>
