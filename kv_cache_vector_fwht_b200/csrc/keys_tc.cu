@@ -608,10 +608,16 @@ __global__ void __launch_bounds__(128, 2)
     }
   }
 
-  // byte offsets, in a chain-ordered row, of this lane's natural channels 4 lane .. 4 lane + 3
-  uint32_t dpos[4];
+  // store round k: this lane's natural channel 4 lane + i_k (i_k from the quantizer's
+  // schedule, so that a round's 32 stores hit 32 banks) to byte offset dpos[k] of the
+  // chain-ordered row, its 2 bytes taken from the lane's 8-byte load by byte permute sel[k]
+  uint32_t dpos[4], sel[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) dpos[i] = 2u * sPos[4 * lane + i];
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t i = tab->gsched[lane][k];
+    dpos[k] = 2u * sPos[4 * lane + i];
+    sel[k] = (2u * i) | ((2u * i + 1u) << 4);
+  }
   // where those channels sit in a staged (swizzled) row: 64-column half lane / 16, 16-byte
   // chunk (lane mod 16) / 2, 8-byte half lane mod 2
   const uint32_t src_off = (lane >> 4) * (kXBuf / 2) + (lane & 1) * 8;
@@ -639,10 +645,9 @@ __global__ void __launch_bounds__(128, 2)
         const int r = warp * 32 + j;
         const uint2 v = *reinterpret_cast<const uint2*>(src + r * 128 + ((src_c ^ static_cast<uint32_t>(r & 7)) << 4));
         uint8_t* dst = sP + r * kGStride;
-        *reinterpret_cast<uint16_t*>(dst + dpos[0]) = static_cast<uint16_t>(v.x);
-        *reinterpret_cast<uint16_t*>(dst + dpos[1]) = static_cast<uint16_t>(v.x >> 16);
-        *reinterpret_cast<uint16_t*>(dst + dpos[2]) = static_cast<uint16_t>(v.y);
-        *reinterpret_cast<uint16_t*>(dst + dpos[3]) = static_cast<uint16_t>(v.y >> 16);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          *reinterpret_cast<uint16_t*>(dst + dpos[k]) = static_cast<uint16_t>(__byte_perm(v.x, v.y, sel[k]));
       }
     }
     mbar_arrive(&bar_free[b]);

@@ -112,6 +112,54 @@ tq_status tq_host_tables(int d, int bits, int mode, uint64_t seed, const int32_t
   return st;
 }
 
+namespace {
+// Store schedule of the grouped kernel's gather (DevTables::gsched). Lane l stores natural
+// channel c = 4l + i to chain position pos[c], a 2-byte slot in bank (pos[c] / 2) mod 32 of a
+// row. Lanes x banks with an edge per (l, i) is a 4-regular bipartite multigraph (each bank
+// holds chain positions 2b, 2b + 1, 2b + 64, 2b + 65), so it splits into 4 perfect matchings
+// (Koenig); each round takes one, found by augmenting paths (Kuhn), and removes it.
+bool gather_augment(int l, const int (&bank)[32][4], const bool (&used)[32][4], bool (&seen)[32],
+                    int (&lane_of_bank)[32], int (&opt_of_lane)[32]) {
+  for (int i = 0; i < 4; ++i) {
+    if (used[l][i]) continue;
+    const int b = bank[l][i];
+    if (seen[b]) continue;
+    seen[b] = true;
+    if (lane_of_bank[b] < 0 ||
+        gather_augment(lane_of_bank[b], bank, used, seen, lane_of_bank, opt_of_lane)) {
+      lane_of_bank[b] = l;
+      opt_of_lane[l] = i;
+      return true;
+    }
+  }
+  return false;
+}
+
+void gather_schedule(const int32_t (&chan)[tq::kD], uint8_t (&sched)[32][4]) {
+  int pos[tq::kD];
+  for (int p = 0; p < tq::kD; ++p) pos[chan[p]] = p;
+  int bank[32][4];
+  for (int l = 0; l < 32; ++l)
+    for (int i = 0; i < 4; ++i) bank[l][i] = (pos[4 * l + i] >> 1) & 31;
+  bool used[32][4] = {};
+  for (int k = 0; k < 4; ++k) {
+    int lane_of_bank[32], opt_of_lane[32];
+    for (int j = 0; j < 32; ++j) lane_of_bank[j] = opt_of_lane[j] = -1;
+    for (int l = 0; l < 32; ++l) {
+      bool seen[32] = {};
+      gather_augment(l, bank, used, seen, lane_of_bank, opt_of_lane);
+    }
+    for (int l = 0; l < 32; ++l) {
+      int i = opt_of_lane[l];
+      if (i < 0)  // cannot happen for a regular multigraph; any unused channel stays correct
+        for (i = 0; used[l][i]; ++i) {}
+      used[l][i] = true;
+      sched[l][k] = static_cast<uint8_t>(i);
+    }
+  }
+}
+}  // namespace
+
 tq_status tq_build_codebook(int d, int bits, int mode, uint64_t seed,
                             const int32_t* outlier_channels, int n_outlier, tq_quantizer** out) {
   if (!out) return TQ_EINVAL;
@@ -162,6 +210,7 @@ tq_status tq_build_codebook(int d, int bits, int mode, uint64_t seed,
         h->s_umma[off] = q->host.s_rot[j * kD + col];
       }
   }
+  if (mode == TQ_MODE_GROUPED) gather_schedule(q->host.chan, h->gsched);
   for (int qq = 0; qq < kD / 2; ++qq)
     h->pair_mask[qq] = (q->host.signs[2 * qq] < 0 ? 1u << 15 : 0u) |
                        (q->host.signs[2 * qq + 1] < 0 ? 1u << 31 : 0u);

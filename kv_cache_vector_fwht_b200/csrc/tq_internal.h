@@ -35,6 +35,10 @@ struct DevTables {
   // rotation signs of bf16 element pairs: word q has bit 15 set if s_{2q} = -1, bit 31 if
   // s_{2q+1} = -1 (an XOR flips both elements of a packed pair).
   alignas(16) uint32_t pair_mask[kD / 2];
+  // grouped: store order of the per-warp gather into chain order. Lane l holds natural
+  // channels 4l .. 4l + 3; in store round k it writes channel 4l + gsched[l][k], chosen so that
+  // the 32 lanes of a round write 32 different shared-memory banks.
+  uint8_t gsched[32][4];
 };
 
 struct HostTables {
