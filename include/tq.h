@@ -182,6 +182,18 @@ tq_status tq_quantize_values(const void* v_dev, int dtype, int64_t n_rows, int64
 tq_status tq_append(const tq_quantizer* q, tq_kv_cache* cache, const void* k_new_dev,
                     const void* v_new_dev, int dtype, int n_tokens, void* stream);
 
+/* One decode step: tq_append of this step's tokens followed by tq_decode_attention, both on
+ * `stream`, launched back to back so that the decode's query prologue overlaps the append
+ * (programmatic dependent launch). Arguments are those of the two calls (k_new_dev /
+ * v_new_dev / kv_dtype / n_tokens for the append; the rest for the decode) and are all
+ * checked before anything is launched; the first error is returned. */
+tq_status tq_append_decode(const tq_quantizer* q, tq_kv_cache* cache, const void* k_new_dev,
+                           const void* v_new_dev, int kv_dtype, int n_tokens,
+                           const void* q_dev, int q_dtype, int n_q_heads,
+                           const int32_t* head_map, float sm_scale, void* out_dev, int out_dtype,
+                           float* scores_dev, int64_t scores_ld,
+                           void* workspace_dev, size_t workspace_bytes, void* stream);
+
 /* Workspace bytes tq_decode_attention needs for this cache and query-head count. The
  * workspace must be zero-filled before its first use; every call leaves it reusable. */
 tq_status tq_decode_workspace_bytes(const tq_kv_cache* cache, int n_q_heads, size_t* bytes);

@@ -29,7 +29,8 @@ D = 128
 
 EXPORTED = ["tq_build_codebook", "tq_free", "tq_key_layout", "tq_host_tables",
             "tq_quantize_keys", "tq_dequantize_keys", "tq_quantize_values", "tq_append", "tq_decode_workspace_bytes",
-            "tq_decode_attention", "tq_decode_attention_noalloc", "tq_decode_attention_partial",
+            "tq_decode_attention", "tq_decode_attention_noalloc", "tq_append_decode",
+            "tq_decode_attention_partial",
             "tq_merge_partials", "tq_set_decode_policy", "tq_sync_status",
             "tq_selftest_bounded_wait", "tq_status_string", "tq_abi_version"]
 
@@ -87,6 +88,10 @@ _lib.tq_decode_attention_noalloc.argtypes = [c_void_p, POINTER(KVCacheDesc), c_v
                                              c_int, POINTER(c_int32), c_float, c_void_p, c_int,
                                              c_void_p, c_int64, c_void_p]
 _lib.tq_decode_attention_noalloc.restype = c_int
+_lib.tq_append_decode.argtypes = [c_void_p, POINTER(KVCacheDesc), c_void_p, c_void_p, c_int, c_int,
+                                  c_void_p, c_int, c_int, POINTER(c_int32), c_float, c_void_p,
+                                  c_int, c_void_p, c_int64, c_void_p, c_size_t, c_void_p]
+_lib.tq_append_decode.restype = c_int
 _lib.tq_decode_attention_partial.argtypes = [c_void_p, POINTER(KVCacheDesc), c_void_p, c_int,
                                              c_int, POINTER(c_int32), c_float, c_void_p,
                                              c_void_p, c_size_t, c_void_p]
@@ -342,6 +347,24 @@ def tq_decode_attention(q: Quantizer, cache: KVCache, query, out=None, workspace
                                     _dtype_code(out) if out is not None else TQ_F32,
                                     _ptr(scores), sld, _ptr(workspace), wbytes, _stream(stream)),
            "tq_decode_attention")
+
+
+def tq_append_decode(q: Quantizer, cache: KVCache, k_new, v_new, query, out=None, workspace=None,
+                     head_map=None, sm_scale: float = 0.0, scores=None, stream=None) -> None:
+    """One decode step: tq_append(k_new, v_new) then tq_decode_attention(query), launched back
+    to back (see tq.h); arguments as for the two calls."""
+    assert k_new.is_contiguous() and k_new.dim() == 4
+    assert query.is_contiguous() and query.dim() == 3
+    hq = query.shape[1]
+    hm = (c_int32 * hq)(*[int(v) for v in head_map]) if head_map is not None else None
+    sld = scores.shape[2] if scores is not None else 0
+    wbytes = workspace.numel() if workspace is not None else 0
+    _check(_lib.tq_append_decode(q.handle, ctypes.byref(cache.desc), _ptr(k_new), _ptr(v_new),
+                                 _dtype_code(k_new), k_new.shape[2], _ptr(query),
+                                 _dtype_code(query), hq, hm, sm_scale, _ptr(out),
+                                 _dtype_code(out) if out is not None else TQ_F32, _ptr(scores),
+                                 sld, _ptr(workspace), wbytes, _stream(stream)),
+           "tq_append_decode")
 
 
 TQ_DECODE_AUTO, TQ_DECODE_ONE_SET, TQ_DECODE_TWO_SETS = 0, 1, 2

@@ -285,8 +285,9 @@ tq_status tq_quantize_values(const void* v, int dtype, int64_t n_rows, int64_t l
                                 static_cast<cudaStream_t>(stream));
 }
 
-tq_status tq_append(const tq_quantizer* q, tq_kv_cache* c, const void* k_new, const void* v_new,
-                    int dtype, int n_tokens, void* stream) {
+// Argument checks of tq_append (nothing launched).
+static tq_status check_append(const tq_quantizer* q, const tq_kv_cache* c, const void* k_new,
+                              const void* v_new, int dtype, int n_tokens) {
   if (!q) return TQ_EINVAL;
   tq_status st = check_cache(q, c);
   if (st != TQ_OK) return st;
@@ -298,6 +299,13 @@ tq_status tq_append(const tq_quantizer* q, tq_kv_cache* c, const void* k_new, co
   if (c->value_bits == 0 && v_new) return TQ_EINVAL;
   for (int b = 0; b < c->batch; ++b)
     if (static_cast<int64_t>(c->len_host[b]) + n_tokens > c->capacity) return TQ_ECAPACITY;
+  return TQ_OK;
+}
+
+tq_status tq_append(const tq_quantizer* q, tq_kv_cache* c, const void* k_new, const void* v_new,
+                    int dtype, int n_tokens, void* stream) {
+  tq_status st = check_append(q, c, k_new, v_new, dtype, n_tokens);
+  if (st != TQ_OK || n_tokens == 0) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (append_fused_ok(q, c, n_tokens)) {
     if ((st = launch_append_fused(q, c, k_new, v_new, dtype, n_tokens, s)) != TQ_OK) return st;
@@ -378,6 +386,28 @@ tq_status tq_decode_attention(const tq_quantizer* q, const tq_kv_cache* c, const
   if (scores && scores_ld < max_len) return TQ_EINVAL;
   if (!workspace || !aligned16(workspace)) return TQ_EINVAL;
   if (workspace_bytes < decode_workspace_bytes(c->batch, n_q_heads, c->capacity)) return TQ_EINVAL;
+  return launch_decode(q, c, qv, q_dtype, n_q_heads, head_map, sm_scale, out, out_dtype, scores,
+                       scores_ld, nullptr, workspace, workspace_bytes,
+                       static_cast<cudaStream_t>(stream));
+}
+
+tq_status tq_append_decode(const tq_quantizer* q, tq_kv_cache* c, const void* k_new,
+                           const void* v_new, int kv_dtype, int n_tokens, const void* qv,
+                           int q_dtype, int n_q_heads, const int32_t* head_map, float sm_scale,
+                           void* out, int out_dtype, float* scores, int64_t scores_ld,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  tq_status st = check_append(q, c, k_new, v_new, kv_dtype, n_tokens);
+  if (st != TQ_OK) return st;
+  if ((st = check_decode_args(q, c, qv, q_dtype, n_q_heads, head_map, out, out_dtype, scores,
+                              scores_ld)) != TQ_OK)
+    return st;
+  if (scores) {  // the scores cover the lengths after the append
+    for (int b = 0; b < c->batch; ++b)
+      if (static_cast<int64_t>(c->len_host[b]) + n_tokens > scores_ld) return TQ_EINVAL;
+  }
+  if (!workspace || !aligned16(workspace)) return TQ_EINVAL;
+  if (workspace_bytes < decode_workspace_bytes(c->batch, n_q_heads, c->capacity)) return TQ_EINVAL;
+  if ((st = tq_append(q, c, k_new, v_new, kv_dtype, n_tokens, stream)) != TQ_OK) return st;
   return launch_decode(q, c, qv, q_dtype, n_q_heads, head_map, sm_scale, out, out_dtype, scores,
                        scores_ld, nullptr, workspace, workspace_bytes,
                        static_cast<cudaStream_t>(stream));

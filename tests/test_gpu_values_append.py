@@ -148,3 +148,43 @@ def test_append_multi_token_chunks(mode, bits, vbits, dtype):
             ref = O.quantize_values(v[b, h].astype(np.float64), vbits)
             assert np.array_equal(cache.v_q[rows].cpu().numpy(), ref["q"])
             assert np.array_equal(cache.v_params[rows].cpu().numpy().view(np.uint16), ref["params"])
+
+
+def test_append_decode_equals_append_then_decode():
+    """tq_append_decode (one call, both kernels launched back to back) leaves the same cache
+    and gives the same outputs and scores, bit for bit, as tq_append followed by
+    tq_decode_attention; a decode argument error launches nothing (lengths unchanged)."""
+    dev = require_cuda()
+    qg = tq.tq_build_codebook(128, 3, "prod", 11)
+    B, H, Hq, cap = 2, 2, 6, 272
+    g = W.rng(12)
+    pre_k = to_device(W.round_bf16(W.scaled_gaussian_rows(g, B * H * 200).reshape(B, H, 200, 128)), torch.bfloat16)
+    pre_v = to_device(W.round_bf16(W.gaussian(g, (B, H, 200, 128))), torch.bfloat16)
+    k_new = to_device(W.round_bf16(W.scaled_gaussian_rows(g, B * H).reshape(B, H, 1, 128)), torch.bfloat16)
+    v_new = to_device(W.round_bf16(W.gaussian(g, (B, H, 1, 128))), torch.bfloat16)
+    q = to_device(W.round_bf16(W.gaussian(g, (B, Hq, 128))), torch.bfloat16)
+    res = []
+    for fused in (False, True):
+        cache = tq.KVCache(qg, B, H, cap, value_bits=2, device=dev)
+        tq.tq_append(qg, cache, pre_k, pre_v)
+        ws = tq.alloc_decode_workspace(cache, Hq)
+        out = torch.empty((B, Hq, 128), device=dev)
+        sc = torch.full((B, Hq, 256), float("nan"), device=dev)
+        if fused:
+            tq.tq_append_decode(qg, cache, k_new, v_new, q, out, ws, scores=sc)
+        else:
+            tq.tq_append(qg, cache, k_new, v_new)
+            tq.tq_decode_attention(qg, cache, q, out, ws, scores=sc)
+        torch.cuda.synchronize()
+        # the written rows only (rows past each length are uninitialised memory)
+        written = lambda t: t.reshape(B * H, cap, -1)[:, :201].cpu()
+        res.append((out.cpu(), sc.cpu(), cache.lengths, written(cache.k_idx), written(cache.v_q)))
+        if fused:
+            with pytest.raises(tq.TQError) as e:   # scores_ld below the post-append length
+                tq.tq_append_decode(qg, cache, k_new, v_new, q, out, ws, scores=sc[:, :, :201])
+            assert e.value.status == tq.TQ_EINVAL
+            assert cache.lengths == [201, 201]
+    (o0, s0, l0, k0, v0), (o1, s1, l1, k1, v1) = res
+    assert l0 == l1 == [201, 201]
+    assert torch.equal(o0, o1) and torch.equal(k0, k1) and torch.equal(v0, v1)
+    assert torch.equal(torch.nan_to_num(s0, nan=-7.0), torch.nan_to_num(s1, nan=-7.0))
