@@ -491,13 +491,8 @@ __global__ void __launch_bounds__(Cfg<NSET>::threads, 1) k_decode(const __grid_c
       }
     }
     __syncthreads();
-    grid_dependency_wait();
-    t1 = min(a.len[b], t0 + a.tokens_per_split);
-    const int c0 = t0 + 32 * warp;
-    if (c0 < t1) {
-      load_keys(c0, kw, sw4, nw);
-      load_values(c0);
-    }
+    // the lookup tables too depend only on the query and the quantizer: built before the
+    // grid-dependency wait, they overlap a preceding append as well
     {
       constexpr int PNI = Lo::PNI, PNS = Lo::PNS, PS = Lo::PS;
       const float* cenI = sCen;        // segment I centroids (grouped: the outlier group)
@@ -604,6 +599,13 @@ __global__ void __launch_bounds__(Cfg<NSET>::threads, 1) k_decode(const __grid_c
       }
     }
     __syncthreads();
+    grid_dependency_wait();
+    t1 = min(a.len[b], t0 + a.tokens_per_split);
+    const int c0 = t0 + 32 * warp;
+    if (c0 < t1) {
+      load_keys(c0, kw, sw4, nw);
+      load_values(c0);
+    }
 
     // ---------------- main loop: this warp's chunks
     // p pairs of the chunk's tokens: sPP[k 32 + token] = ((p_2k, p_2k), (p_2k+1, p_2k+1))
