@@ -25,7 +25,7 @@ Sources (page title, section):
              (codebook MSE), Theorem 2 (unbiasedness), Theorem 3 (distortion), recall,
              rank correlation, needle and compression checks; value_bits / group_size 32.
 
-Readings where the pages are silent are stated at each function (see also DESIGN.md).
+Readings where the pages are silent are stated at each function.
 Parity pins: every public function here is pinned by tests/test_oracle_*.py.
 """
 from __future__ import annotations
