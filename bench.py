@@ -52,6 +52,23 @@ def value_bytes(vb):
     return 128 * vb // 8 + 16
 
 
+WL_DESC = {"decode-s": "decode-s: batch 1, 12 q heads / 2 kv heads, d 128, ctx 32768, "
+                       "keys 3-bit prod, values 2-bit g32",
+           "decode-l": "decode-l: batch 8, 28 q heads / 4 kv heads, d 128, ctx 32768, "
+                       "keys 3-bit prod, values 2-bit g32",
+           "decode-stream": "decode-stream: batch 1, 64 q heads / 8 kv heads, d 128, "
+                            "ctx 131072, keys 4-bit prod, values 4-bit g32"}
+
+
+def decode_config(name: str, world: int) -> dict:
+    """The `config` of a decode workload's JSON line (both arms)."""
+    wl = DECODE_WORKLOADS[name]
+    return {"workload": WL_DESC[name], "global_batch": wl["batch"] * world, "seq_len": wl["ctx"],
+            "parallelism": f"replicas x{world}",
+            "data_types": "bf16 query and new K/V rows, u8 packed cache, fp16 norms and value "
+                          "params (the arithmetic type is the line's dtype)"}
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -334,12 +351,6 @@ def run_tq(args):
     nh_cta = -(-heads_per_kv // -(-heads_per_kv // cap))   # query heads per block
     nh_tpl = (2 if nh_cta <= 2 else nh_cta) if not two_sets else (6 if nh_cta <= 6 else 8)
     n_sets = 2 if two_sets else 1
-    wl_desc = {"decode-s": "decode-s: batch 1, 12 q heads / 2 kv heads, d 128, ctx 32768, "
-                           "keys 3-bit prod, values 2-bit g32",
-               "decode-l": "decode-l: batch 8, 28 q heads / 4 kv heads, d 128, ctx 32768, "
-                           "keys 3-bit prod, values 2-bit g32",
-               "decode-stream": "decode-stream: batch 1, 64 q heads / 8 kv heads, d 128, "
-                                "ctx 131072, keys 4-bit prod, values 4-bit g32"}[args.decode_workload]
     result = {
         "metric": f"fused-decode keys scored/s ({args.decode_workload} step: append 1 token per "
                   "KV head + decode)",
@@ -347,11 +358,8 @@ def run_tq(args):
         "ms_per_step": tot_ms_max / steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded torch CUDA generator; N(0,1) x U[2,20] keys)",
-        "config": {"workload": wl_desc,
-                   "global_batch": B * world, "seq_len": N, "parallelism": f"replicas x{world}",
-                   "data_types": "bf16 query and new K/V rows, u8 packed cache, fp16 norms "
-                                 "and value params, fp32 arithmetic",
-                   "l2": "flushed (256 MiB write) before each step, outside its events"},
+        "config": dict(decode_config(args.decode_workload, world),
+                       l2="flushed (256 MiB write) before each step, outside its events"),
         "decode_gbs": achieved,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": None,
@@ -509,7 +517,7 @@ def run_reference(args):
         "token per KV head + decode)", "value": value, "unit": "keys/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": "decode-s (sampled context)"},
+        "data": "synthetic", "config": decode_config("decode-s", args.gpus),
         "cpu_baseline": {"value": value, "unit": "keys/s", "cores": _cores(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "keys/s", "h2d_bytes_per_step": 0,
