@@ -126,6 +126,15 @@ tq_status tq_build_codebook(int d, int bits, int mode, uint64_t seed,
                             const int32_t* outlier_channels, int n_outlier,
                             tq_quantizer** out);
 
+/* The same quantizer without a device copy of its tables, built on the host alone (no GPU
+ * needed): for plane sizes (tq_key_layout) and for checking arguments before device memory
+ * exists. Every device entry point given it runs its argument checks (and returns their
+ * errors) and then returns TQ_ECUDA without launching anything or changing the cache.
+ * Free it with tq_free. Errors as tq_build_codebook (no TQ_ECUDA). */
+tq_status tq_build_codebook_host(int d, int bits, int mode, uint64_t seed,
+                                 const int32_t* outlier_channels, int n_outlier,
+                                 tq_quantizer** out);
+
 void tq_free(tq_quantizer* q);
 
 /* Plane sizes of a quantizer's keys (host only). */
@@ -183,10 +192,15 @@ tq_status tq_append(const tq_quantizer* q, tq_kv_cache* cache, const void* k_new
                     const void* v_new_dev, int dtype, int n_tokens, void* stream);
 
 /* One decode step: tq_append of this step's tokens followed by tq_decode_attention, both on
- * `stream`, launched back to back so that the decode's query prologue overlaps the append
- * (programmatic dependent launch). Arguments are those of the two calls (k_new_dev /
- * v_new_dev / kv_dtype / n_tokens for the append; the rest for the decode) and are all
- * checked before anything is launched; the first error is returned. */
+ * `stream`. The decode is launched with programmatic dependent launch right behind the
+ * library's own append kernel, so that its query-only prologue (query rotation, S q, lookup
+ * tables) overlaps the append; it reads the lengths and the cache only once the append has
+ * completed. The query must be ready when this call's first kernel starts (written by work
+ * ordered before the call on `stream`), which stream order already guarantees. Arguments are
+ * those of the two calls (k_new_dev / v_new_dev / kv_dtype / n_tokens for the append; the
+ * rest for the decode) and are all checked before anything is launched, including the
+ * decode's head grouping for the lengths after the append: on any error nothing is launched
+ * and the cache is unchanged; the first error is returned. */
 tq_status tq_append_decode(const tq_quantizer* q, tq_kv_cache* cache, const void* k_new_dev,
                            const void* v_new_dev, int kv_dtype, int n_tokens,
                            const void* q_dev, int q_dtype, int n_q_heads,
@@ -204,9 +218,8 @@ tq_status tq_decode_workspace_bytes(const tq_kv_cache* cache, int n_q_heads, siz
  *   mse:     s_i = ||x_i|| <Pi q, c[idx_i]>
  *   grouped: s_i = sum over the two channel groups g of ||x_i,g|| <Pi_g q_g, c_g[idx_i,g]>
  *   out = softmax(sm_scale * s) . v_hat,   v_hat = mn16 + code * s16.
- * The kernel is launched with programmatic dependent launch: after tq_append on the same
- * stream its query-only prologue overlaps the append kernel; it reads the lengths and the
- * cache only once the preceding kernels have completed.
+ * The kernel is an ordinary launch on `stream`: every earlier work on the stream (the query's
+ * producer included) has completed when it starts.
  * q_dev: batch x n_q_heads x d (TQ_F32 or TQ_BF16). head_map: host int32[n_q_heads] with
  * values in [0, n_kv_heads), NULL = h / (n_q_heads / n_kv_heads). sm_scale <= 0 means
  * 1/sqrt(d). out_dev: batch x n_q_heads x d in out_dtype (TQ_F32 or TQ_BF16), may be NULL
@@ -244,19 +257,18 @@ tq_status tq_decode_attention_noalloc(const tq_quantizer* q, const tq_kv_cache* 
 
 /* Shape of the fused decode's thread blocks (process-wide; a tuning and testing knob, the
  * results do not depend on it beyond fp32 rounding order). A block scores and sums the
- * tokens of one KV head for a group of its query heads. TQ_DECODE_AUTO (the default): groups
- * of up to 8 query heads (two 4-head lookup-table sets, 12 warps) when a KV head has more
- * than 4 and the decode holds at least 4 x 384 (token, KV head) units per SM, else groups of
- * up to 4 (one table set, 16 warps). TQ_DECODE_ONE_SET and TQ_DECODE_TWO_SETS force one
- * shape (two sets only where a KV head has more than 4 query heads and the two-set tables
- * fit the shared memory; grouped keys always use one set). Writes the previous policy to
- * `previous` (nullable); TQ_EINVAL for another value (nothing changed). */
+ * tokens of one KV head for a group of its query heads. TQ_DECODE_AUTO (the default) and
+ * TQ_DECODE_TWO_SETS: groups of up to 8 query heads (two 4-head lookup-table sets, 8 warps)
+ * when a KV head has more than 4 and the two-set tables fit the shared memory, else groups
+ * of up to 4 (one table set, 16 warps); grouped keys always use one set. TQ_DECODE_ONE_SET
+ * forces groups of up to 4. Writes the previous policy to `previous` (nullable); TQ_EINVAL
+ * for another value (nothing changed). */
 #define TQ_DECODE_AUTO 0
 #define TQ_DECODE_ONE_SET 1
 #define TQ_DECODE_TWO_SETS 2
 tq_status tq_set_decode_policy(int policy, int* previous);
 
-/* ---- context-parallel decode/* ---- context-parallel decode (a cache's context split into slices, e.g. one per GPU) ----
+/* ---- context-parallel decode (a cache's context split into slices, e.g. one per GPU) ----
  * Softmax attention over the union of the slices equals the LSE merge of per-slice partial
  * results (the merge the fused decode kernel already runs between its own context splits):
  *   step 1, per slice:  tq_decode_attention_partial -> (m, l, o) per (sequence, query head)

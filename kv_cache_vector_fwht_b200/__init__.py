@@ -27,7 +27,7 @@ MODES = {"mse": 0, "prod": 1, "grouped": 2}
 TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 D = 128
 
-EXPORTED = ["tq_build_codebook", "tq_free", "tq_key_layout", "tq_host_tables",
+EXPORTED = ["tq_build_codebook", "tq_build_codebook_host", "tq_free", "tq_key_layout", "tq_host_tables",
             "tq_quantize_keys", "tq_dequantize_keys", "tq_quantize_values", "tq_append", "tq_decode_workspace_bytes",
             "tq_decode_attention", "tq_decode_attention_noalloc", "tq_append_decode",
             "tq_decode_attention_partial",
@@ -58,6 +58,9 @@ class KVCacheDesc(ctypes.Structure):
 _lib.tq_build_codebook.argtypes = [c_int, c_int, c_int, c_uint64, POINTER(c_int32), c_int,
                                    POINTER(c_void_p)]
 _lib.tq_build_codebook.restype = c_int
+_lib.tq_build_codebook_host.argtypes = [c_int, c_int, c_int, c_uint64, POINTER(c_int32), c_int,
+                                        POINTER(c_void_p)]
+_lib.tq_build_codebook_host.restype = c_int
 _lib.tq_free.argtypes = [c_void_p]
 _lib.tq_free.restype = None
 _lib.tq_key_layout.argtypes = [c_void_p, POINTER(KeyLayout)]
@@ -228,6 +231,16 @@ def tq_build_codebook(d: int, bits: int, mode: str, seed: int, outliers=None) ->
     out_arr, n_out = _outlier_arg(outliers)
     _check(_lib.tq_build_codebook(d, bits, MODES[mode], seed, out_arr, n_out, ctypes.byref(h)),
            "tq_build_codebook")
+    return Quantizer(h.value, d, bits, mode, seed)
+
+
+def tq_build_codebook_host(d: int, bits: int, mode: str, seed: int, outliers=None) -> Quantizer:
+    """A quantizer without device tables (no GPU needed): plane sizes and argument checks;
+    device entry points given it return TQ_ECUDA after their checks (see tq.h)."""
+    h = c_void_p()
+    out_arr, n_out = _outlier_arg(outliers)
+    _check(_lib.tq_build_codebook_host(d, bits, MODES[mode], seed, out_arr, n_out,
+                                       ctypes.byref(h)), "tq_build_codebook_host")
     return Quantizer(h.value, d, bits, mode, seed)
 
 

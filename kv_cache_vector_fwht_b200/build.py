@@ -17,9 +17,10 @@ OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libtq.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
-SOURCES = ["tq_api.cu", "quantize.cu", "keys_tc.cu", "dequant.cu", "decode.cu", "append.cu",
+SOURCES = ["tq_api.cu", "quantize.cu", "keys_tc.cu", "dequant.cu", "decode.cu", "decode_prod.cu",
+           "decode_mse.cu", "decode_grp.cu", "append.cu",
            "tq_host.cpp"]
-HEADERS = ["tq_internal.h", "tq_device.cuh", os.path.join("..", "..", "include", "tq.h")]
+HEADERS = ["tq_internal.h", "tq_device.cuh", "decode_kernel.cuh", os.path.join("..", "..", "include", "tq.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O3",
          "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]

@@ -160,8 +160,9 @@ void gather_schedule(const int32_t (&chan)[tq::kD], uint8_t (&sched)[32][4]) {
 }
 }  // namespace
 
-tq_status tq_build_codebook(int d, int bits, int mode, uint64_t seed,
-                            const int32_t* outlier_channels, int n_outlier, tq_quantizer** out) {
+static tq_status build_quantizer(int d, int bits, int mode, uint64_t seed,
+                                 const int32_t* outlier_channels, int n_outlier, bool device,
+                                 tq_quantizer** out) {
   if (!out) return TQ_EINVAL;
   *out = nullptr;
   tq_quantizer* q = new (std::nothrow) tq_quantizer;
@@ -177,6 +178,11 @@ tq_status tq_build_codebook(int d, int bits, int mode, uint64_t seed,
   q->bits = bits;
   q->mode = mode;
   q->seed = seed;
+  q->device = -1;
+  if (!device) {  // host-only: layouts and argument checks, no device tables
+    *out = q;
+    return TQ_OK;
+  }
 
   DevTables* h = new (std::nothrow) DevTables;
   if (!h) {
@@ -235,6 +241,17 @@ tq_status tq_build_codebook(int d, int bits, int mode, uint64_t seed,
   return TQ_OK;
 }
 
+tq_status tq_build_codebook(int d, int bits, int mode, uint64_t seed,
+                            const int32_t* outlier_channels, int n_outlier, tq_quantizer** out) {
+  return build_quantizer(d, bits, mode, seed, outlier_channels, n_outlier, true, out);
+}
+
+tq_status tq_build_codebook_host(int d, int bits, int mode, uint64_t seed,
+                                 const int32_t* outlier_channels, int n_outlier,
+                                 tq_quantizer** out) {
+  return build_quantizer(d, bits, mode, seed, outlier_channels, n_outlier, false, out);
+}
+
 void tq_free(tq_quantizer* q) {
   if (!q) return;
   if (q->dev) cudaFree(q->dev);
@@ -255,6 +272,7 @@ tq_status tq_quantize_keys(const tq_quantizer* q, const void* x, int dtype, int6
   if (n_rows == 0) return TQ_OK;
   if ((st = check_key_planes(q, out)) != TQ_OK) return st;
   if (q->mode != TQ_MODE_GROUPED && (reinterpret_cast<uintptr_t>(out.norms) & 3u)) return TQ_EINVAL;
+  if (!q->dev) return TQ_ECUDA;
   return launch_quantize_keys(q, x, dtype, n_rows, ld, out, RowMap{nullptr, 0, 0, 0},
                               static_cast<cudaStream_t>(stream));
 }
@@ -266,6 +284,7 @@ tq_status tq_dequantize_keys(const tq_quantizer* q, tq_key_planes planes, int64_
   if (st != TQ_OK) return st;
   if (n_rows == 0) return TQ_OK;
   if ((st = check_key_planes(q, planes)) != TQ_OK) return st;
+  if (!q->dev) return TQ_ECUDA;
   return launch_dequantize_keys(q, planes, n_rows, out, out_dtype, ld,
                                 static_cast<cudaStream_t>(stream));
 }
@@ -306,6 +325,7 @@ tq_status tq_append(const tq_quantizer* q, tq_kv_cache* c, const void* k_new, co
                     int dtype, int n_tokens, void* stream) {
   tq_status st = check_append(q, c, k_new, v_new, dtype, n_tokens);
   if (st != TQ_OK || n_tokens == 0) return st;
+  if (!q->dev) return TQ_ECUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (append_fused_ok(q, c, n_tokens)) {
     if ((st = launch_append_fused(q, c, k_new, v_new, dtype, n_tokens, s)) != TQ_OK) return st;
@@ -330,8 +350,7 @@ tq_status tq_decode_workspace_bytes(const tq_kv_cache* c, int n_q_heads, size_t*
   return TQ_OK;
 }
 
-// Argument checks of the no-workspace decode entry point (the same as tq_decode_attention's
-// checks apart from the workspace).
+// Argument checks of every decode entry point (the workspace apart: check_workspace).
 static tq_status check_decode_args(const tq_quantizer* q, const tq_kv_cache* c, const void* qv,
                                    int q_dtype, int n_q_heads, const int32_t* head_map,
                                    void* out, int out_dtype, float* scores, int64_t scores_ld) {
@@ -359,35 +378,23 @@ static tq_status check_decode_args(const tq_quantizer* q, const tq_kv_cache* c, 
   return TQ_OK;
 }
 
+static tq_status check_workspace(const tq_kv_cache* c, int n_q_heads, const void* workspace,
+                                 size_t workspace_bytes) {
+  if (!workspace || !aligned16(workspace)) return TQ_EINVAL;
+  if (workspace_bytes < decode_workspace_bytes(c->batch, n_q_heads, c->capacity)) return TQ_EINVAL;
+  return TQ_OK;
+}
+
 tq_status tq_decode_attention(const tq_quantizer* q, const tq_kv_cache* c, const void* qv,
                               int q_dtype, int n_q_heads, const int32_t* head_map, float sm_scale,
                               void* out, int out_dtype, float* scores, int64_t scores_ld,
                               void* workspace, size_t workspace_bytes, void* stream) {
-  if (!q) return TQ_EINVAL;
-  tq_status st = check_cache(q, c);
+  tq_status st = check_decode_args(q, c, qv, q_dtype, n_q_heads, head_map, out, out_dtype,
+                                   scores, scores_ld);
   if (st != TQ_OK) return st;
-  if (n_q_heads <= 0 || n_q_heads > 512) return TQ_EINVAL;
-  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_EUNSUPPORTED;
-  if (!qv || !aligned16(qv)) return TQ_EINVAL;
-  if (head_map) {
-    for (int h = 0; h < n_q_heads; ++h)
-      if (head_map[h] < 0 || head_map[h] >= c->n_kv_heads) return TQ_EINVAL;
-  } else if (n_q_heads % c->n_kv_heads != 0) {
-    return TQ_EINVAL;
-  }
-  if (c->value_bits != 0) {
-    if (!out || !aligned16(out)) return TQ_EINVAL;
-    if (out_dtype != TQ_F32 && out_dtype != TQ_BF16) return TQ_EUNSUPPORTED;
-  } else if (out) {
-    return TQ_EINVAL;
-  }
-  int max_len = 0;
-  for (int b = 0; b < c->batch; ++b) max_len = c->len_host[b] > max_len ? c->len_host[b] : max_len;
-  if (scores && scores_ld < max_len) return TQ_EINVAL;
-  if (!workspace || !aligned16(workspace)) return TQ_EINVAL;
-  if (workspace_bytes < decode_workspace_bytes(c->batch, n_q_heads, c->capacity)) return TQ_EINVAL;
+  if ((st = check_workspace(c, n_q_heads, workspace, workspace_bytes)) != TQ_OK) return st;
   return launch_decode(q, c, qv, q_dtype, n_q_heads, head_map, sm_scale, out, out_dtype, scores,
-                       scores_ld, nullptr, workspace, workspace_bytes,
+                       scores_ld, nullptr, workspace, workspace_bytes, /*pdl=*/false,
                        static_cast<cudaStream_t>(stream));
 }
 
@@ -405,11 +412,16 @@ tq_status tq_append_decode(const tq_quantizer* q, tq_kv_cache* c, const void* k_
     for (int b = 0; b < c->batch; ++b)
       if (static_cast<int64_t>(c->len_host[b]) + n_tokens > scores_ld) return TQ_EINVAL;
   }
-  if (!workspace || !aligned16(workspace)) return TQ_EINVAL;
-  if (workspace_bytes < decode_workspace_bytes(c->batch, n_q_heads, c->capacity)) return TQ_EINVAL;
+  if ((st = check_workspace(c, n_q_heads, workspace, workspace_bytes)) != TQ_OK) return st;
+  // the decode's head grouping is checked before the append, so that an error leaves the
+  // cache as it was
+  if ((st = check_decode_plan(q, c, n_q_heads, head_map, n_tokens)) != TQ_OK) return st;
+  if (!q->dev) return TQ_ECUDA;
   if ((st = tq_append(q, c, k_new, v_new, kv_dtype, n_tokens, stream)) != TQ_OK) return st;
+  // the kernel just launched is the library's append, ordered after the query's producer:
+  // the decode may start its query-only prologue while the append runs
   return launch_decode(q, c, qv, q_dtype, n_q_heads, head_map, sm_scale, out, out_dtype, scores,
-                       scores_ld, nullptr, workspace, workspace_bytes,
+                       scores_ld, nullptr, workspace, workspace_bytes, /*pdl=*/true,
                        static_cast<cudaStream_t>(stream));
 }
 
@@ -424,10 +436,10 @@ tq_status tq_decode_attention_partial(const tq_quantizer* q, const tq_kv_cache* 
   tq_status st = check_decode_args(q, c, qv, q_dtype, n_q_heads, head_map, part, TQ_F32,
                                    nullptr, 0);
   if (st != TQ_OK) return st;
-  if (!workspace || !aligned16(workspace)) return TQ_EINVAL;
-  if (workspace_bytes < decode_workspace_bytes(c->batch, n_q_heads, c->capacity)) return TQ_EINVAL;
+  if ((st = check_workspace(c, n_q_heads, workspace, workspace_bytes)) != TQ_OK) return st;
   return launch_decode(q, c, qv, q_dtype, n_q_heads, head_map, sm_scale, nullptr, TQ_F32, nullptr,
-                       0, part, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+                       0, part, workspace, workspace_bytes, /*pdl=*/false,
+                       static_cast<cudaStream_t>(stream));
 }
 
 tq_status tq_set_decode_policy(int policy, int* previous) {
@@ -449,9 +461,11 @@ tq_status tq_decode_attention_noalloc(const tq_quantizer* q, const tq_kv_cache* 
                                       const int32_t* head_map, float sm_scale, void* out,
                                       int out_dtype, float* scores, int64_t scores_ld,
                                       void* stream) {
-  const tq_status st = check_decode_args(q, c, qv, q_dtype, n_q_heads, head_map, out, out_dtype,
-                                         scores, scores_ld);
+  tq_status st = check_decode_args(q, c, qv, q_dtype, n_q_heads, head_map, out, out_dtype,
+                                   scores, scores_ld);
   if (st != TQ_OK) return st;
+  if ((st = check_decode_plan(q, c, n_q_heads, head_map, 0)) != TQ_OK) return st;
+  if (!q->dev) return TQ_ECUDA;
   return launch_decode_noalloc(q, c, qv, q_dtype, n_q_heads, head_map, sm_scale, out, out_dtype,
                                scores, scores_ld, static_cast<cudaStream_t>(stream));
 }

@@ -101,18 +101,18 @@ bool append_fused_ok(const tq_quantizer* q, const tq_kv_cache* c, int n_tokens);
 tq_status launch_append_fused(const tq_quantizer* q, tq_kv_cache* c, const void* k_new,
                               const void* v_new, int dtype, int n_tokens, cudaStream_t st);
 
-struct DecodePlan {
-  int n_groups;          // CTA head groups over all KV heads
-  int n_splits;          // context splits per (sequence, head group)
-  int tokens_per_split;  // multiple of 32
-  int max_len;
-};
-
 size_t decode_workspace_bytes(int batch, int n_q_heads, int capacity);
+// Fused decode; pdl: launch with programmatic dependent launch (only right after the
+// library's own append kernel, which was itself ordered after the query's producer).
 tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* cache, const void* qv,
                         int q_dtype, int n_q_heads, const int32_t* head_map, float sm_scale,
                         void* out, int out_dtype, float* scores, int64_t scores_ld,
-                        float* part_out, void* workspace, size_t workspace_bytes, cudaStream_t st);
+                        float* part_out, void* workspace, size_t workspace_bytes, bool pdl,
+                        cudaStream_t st);
+// The head grouping of a decode over the cache's lengths plus len_add tokens, without
+// launching: TQ_EUNSUPPORTED when it needs more head groups than one launch holds.
+tq_status check_decode_plan(const tq_quantizer* q, const tq_kv_cache* cache, int n_q_heads,
+                            const int32_t* head_map, int len_add);
 tq_status set_decode_policy(int policy, int* previous);
 tq_status launch_merge_partials(const float* parts, int n_parts, int64_t rows, void* out,
                                 int out_dtype, cudaStream_t st);
