@@ -257,10 +257,11 @@ tq_status tq_decode_attention_noalloc(const tq_quantizer* q, const tq_kv_cache* 
 
 /* Shape of the fused decode's thread blocks (process-wide; a tuning and testing knob, the
  * results do not depend on it beyond fp32 rounding order). A block scores and sums the
- * tokens of one KV head for a group of its query heads. TQ_DECODE_AUTO (the default) and
- * TQ_DECODE_TWO_SETS: groups of up to 8 query heads (two 4-head lookup-table sets, 8 warps)
- * when a KV head has more than 4 and the two-set tables fit the shared memory, else groups
- * of up to 4 (one table set, 16 warps); grouped keys always use one set. TQ_DECODE_ONE_SET
+ * tokens of one KV head for a group of its query heads. TQ_DECODE_AUTO (the default): groups
+ * of up to 8 query heads (two 4-head lookup-table sets, 8 warps) when a KV head has more
+ * than 4, the two-set tables fit the shared memory and the decode holds at least 4 x 256
+ * (token, KV head) units per SM; else groups of up to 4 (one table set, 16 warps). Grouped
+ * keys always use one set. TQ_DECODE_TWO_SETS drops the size condition; TQ_DECODE_ONE_SET
  * forces groups of up to 4. Writes the previous policy to `previous` (nullable); TQ_EINVAL
  * for another value (nothing changed). */
 #define TQ_DECODE_AUTO 0

@@ -112,11 +112,17 @@ tq_status plan_decode(const tq_quantizer* q, const tq_kv_cache* c, int n_q_heads
       per_kv_max = std::max(per_kv_max, ++seen_n[i]);
     }
   }
-  // Blocks of up to 8 query heads (two table sets) when some KV head has more than 4 and
-  // the two-set layout fits; tq_set_decode_policy can force either shape.
+  // Blocks of up to 8 query heads (two table sets) when some KV head has more than 4, the
+  // two-set layout fits, and the decode is large enough to amortise the two-set block's
+  // longer fixed path (twice the tables to build, more heads per chunk): at least 4 chunk
+  // rounds of (token, KV head) units per SM. Measured: 1.05 M units (batch 8 x 4 KV heads x
+  // 32768, or 1 x 8 x 131072) run 15-20 % faster with two sets; 65536 units (1 x 2 x 32768)
+  // run 15 % slower. tq_set_decode_policy can force either shape.
   const int policy = g_decode_policy.load(std::memory_order_relaxed);
+  const long long units = static_cast<long long>(c->batch) * c->n_kv_heads * max_len;
   p->two = per_kv_max > kSetHeads && two_sets_ok(p->kind, p->mb, p->vb) &&
-           policy != TQ_DECODE_ONE_SET;
+           policy != TQ_DECODE_ONE_SET &&
+           (policy == TQ_DECODE_TWO_SETS || units >= 4ll * Shape<2>::chunk_stride * sms);
   const int cap = p->two ? kMaxSlots : kSetHeads;
 
   // head groups: the query heads of each KV head, in balanced groups of at most `cap`
@@ -220,6 +226,7 @@ tq_status launch_decode(const tq_quantizer* q, const tq_kv_cache* c, const void*
   a.scores = scores;
   a.scores_ld = scores_ld;
   a.tab = q->dev;
+  a.err = device_error_word();
   a.n_kv_heads = c->n_kv_heads;
   a.capacity = c->capacity;
   a.n_q_heads = n_q_heads;

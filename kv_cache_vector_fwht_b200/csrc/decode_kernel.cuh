@@ -78,6 +78,7 @@ struct DecodeArgs {
   float* part_out;  // nullable: per (sequence, query head) (m, l, o) records instead of out
   float* part;
   int* counters;
+  int* err;         // device error word (bounded waits that ran out); see tq_sync_status
   const DevTables* tab;
   int64_t scores_ld;
   int n_kv_heads, capacity, n_q_heads;
@@ -318,6 +319,324 @@ __device__ __forceinline__ void build_table(uint8_t* lut, const float* x, int c0
 // K = kMse: s = n16 <Pi q, c[idx]>; kProd: + r16 sqrt(pi/2)/d <S q, 2 sigma - 1>;
 // kGrp: s = n_o <Pi_o q_o, c_o[idx_o]> + n_n <Pi_n q_n, c_n[idx_n]> over the two channel
 // groups (Pi_g: 32-point Hadamard blocks after the group's signs).
+// L2 prefetch of the packed rows of one 32-token chunk starting at ts (tokens below tp1):
+// the index, sign, norm, value-code and value-parameter planes, one 128-byte line a lane.
+template <int IB, int NB, int VQB, bool PROD, bool HAS_V>
+__device__ __forceinline__ void prefetch_rows(const DecodeArgs& a, int64_t kvrow, int ts, int tp1,
+                                              int lane) {
+  const int n = min(32, tp1 - ts);
+  if (n <= 0) return;
+  const uint8_t* rng[5] = {a.k_idx + (kvrow + ts) * IB, a.k_sgn + (kvrow + ts) * 16,
+                           reinterpret_cast<const uint8_t*>(a.k_nrm) + (kvrow + ts) * NB,
+                           a.v_q + (kvrow + ts) * VQB,
+                           reinterpret_cast<const uint8_t*>(a.v_par) + (kvrow + ts) * 16};
+  const int len_b[5] = {n * IB, PROD ? n * 16 : 0, n * NB, HAS_V ? n * VQB : 0, HAS_V ? n * 16 : 0};
+#pragma unroll
+  for (int r = 0; r < 5; ++r)
+    for (int o = lane * 128; o < len_b[r]; o += 32 * 128)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(rng[r] + o));
+}
+
+// The query prologue of a block (it reads only the query and the quantizer's tables): q_rot =
+// H (s . q) per head slot (grouped: gathered in channel order, 32-point blocks), Sq = S_rot
+// q_rot / sqrt(d) on tensor cores (mma.sync, fp16 hi + lo halves of q_rot, fp32 accumulation),
+// then the byte lookup tables of every set. Every thread of the block takes part; the block
+// has at least 8 warps. Ends with the tables complete (a block-wide barrier).
+template <class Lo, int K, int NSET, int NT>
+__device__ __forceinline__ void decode_prologue(const DecodeArgs& a, uint8_t* smem, float* sCen,
+                                                const int16_t* gheads, int nh, int b) {
+  constexpr int SL = Lo::SL, PI = Lo::PI;
+  constexpr bool PROD = K == kProd, GRP = K == kGrp;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint8_t* lutI = smem + Lo::lutI;
+  uint8_t* lutS = smem + Lo::lutS;
+  float* qrT = reinterpret_cast<float*>(smem + Lo::qrT);
+  float* sqT = reinterpret_cast<float*>(smem + Lo::sqT);
+  uint8_t* qhi = smem + Lo::qhi;
+  uint8_t* qlo = smem + Lo::qlo;
+  float* qinv = reinterpret_cast<float*>(smem + Lo::qinv);
+  const DevTables* __restrict__ tab = a.tab;
+  // S_rot rows [16 warp, 16 warp + 16) as mma.sync A fragments (warps 0..7)
+  uint32_t afr[8][4];
+  if (PROD && warp < 8) {
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t* r0 = reinterpret_cast<const uint32_t*>(tab->s_rot + (16 * warp + g) * kD);
+    const uint32_t* r1 = r0 + 8 * kD / 2;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      afr[kk][0] = __ldg(r0 + kk * 8 + t);
+      afr[kk][1] = __ldg(r1 + kk * 8 + t);
+      afr[kk][2] = __ldg(r0 + kk * 8 + 4 + t);
+      afr[kk][3] = __ldg(r1 + kk * 8 + 4 + t);
+    }
+  }
+  if (warp < 8) {
+    // q_rot of head slot `warp` (zeros for empty slots): signs, then the 128-point
+    // transform with 4 values per lane (2 stages in registers, 5 across lanes)
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (warp < nh) {
+      const int hq = gheads[warp];
+      const int64_t qoff = (static_cast<int64_t>(b) * a.n_q_heads + hq) * kD;
+      if constexpr (GRP) {
+        // chain order: the outlier channels, then the normal channels
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int c = tab->chan[4 * lane + i];
+          v[i] = a.q_f32 ? static_cast<const float*>(a.q)[qoff + c]
+                         : __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t*>(a.q)[qoff + c]) << 16);
+        }
+      } else {
+        if (a.q_f32) load4<true>(static_cast<const float*>(a.q) + qoff, 4 * lane, v);
+        else load4<false>(static_cast<const uint16_t*>(a.q) + qoff, 4 * lane, v);
+      }
+      const uint32_t sw = tab->sign_bits[lane >> 3];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = flip_sign(v[i], sw, (4 * lane + i) & 31);
+      // 128-point transform; grouped: 32-point blocks (lanes 8k .. 8k + 7)
+      fwht_reg<4>(v);
+#pragma unroll
+      for (int mm = 1; mm < (GRP ? 8 : 32); mm <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float other = __shfl_xor_sync(kFull, v[i], mm);
+          v[i] = (lane & mm) ? (other - v[i]) : (v[i] + other);
+        }
+      }
+    }
+    // power-of-two scale so the fp16 hi/lo split neither overflows nor underflows
+    float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+    amax = warp_max(amax);
+    const uint32_t ex = (__float_as_uint(amax) >> 23) & 0xffu;
+    const bool big = ex >= 12u;
+    const float scl = big ? __uint_as_float((264u - ex) << 23) : 1.f;
+    const float inv = big ? __uint_as_float((ex - 10u) << 23) : 1.f;
+    if (lane == 0) qinv[warp] = inv;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = 4 * lane + i;
+      if (warp < SL) qrT[j * SL + warp] = v[i];
+      const float sv = v[i] * scl;
+      const __half hi = __float2half_rn(sv);
+      const __half lo = __float2half_rn(sv - __half2float(hi));
+      reinterpret_cast<__half*>(qhi + warp * kQStride)[j] = hi;
+      reinterpret_cast<__half*>(qlo + warp * kQStride)[j] = lo;
+    }
+  }
+  if (threadIdx.x < 32) sCen[threadIdx.x] = (&tab->cent[0][0])[threadIdx.x];
+  __syncthreads();
+  if (PROD && warp < 8) {
+    // Sq = S_rot q_rot / sqrt(d) for the head slots on tensor cores: mma.sync m16n8k16
+    // (fp16 S_rot is exact; q_rot enters as hi + lo fp16 halves; fp32 accumulation).
+    const int g = lane >> 2, t = lane & 3;
+    float c0 = 0.f, c1 = 0.f, c2 = 0.f, c3 = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const int k0 = 16 * kk;
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const uint8_t* bq = (part ? qlo : qhi) + g * kQStride;
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(bq + (k0 + 2 * t) * 2);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(bq + (k0 + 8 + 2 * t) * 2);
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+            "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};\n"
+            : "+f"(c0), "+f"(c1), "+f"(c2), "+f"(c3)
+            : "r"(afr[kk][0]), "r"(afr[kk][1]), "r"(afr[kk][2]), "r"(afr[kk][3]), "r"(b0), "r"(b1));
+      }
+    }
+    if (2 * t < SL) {  // columns 2t, 2t + 1 are head slots
+      const float s0 = qinv[2 * t] * 0.088388347648318440550f;      // / sqrt(128)
+      const float s1 = qinv[2 * t + 1] * 0.088388347648318440550f;
+      const int j0 = 16 * warp + g;
+      sqT[j0 * SL + 2 * t] = c0 * s0;
+      sqT[j0 * SL + 2 * t + 1] = c1 * s1;
+      sqT[(j0 + 8) * SL + 2 * t] = c2 * s0;
+      sqT[(j0 + 8) * SL + 2 * t + 1] = c3 * s1;
+    }
+  }
+  if constexpr (PROD) __syncthreads();
+  {
+    // entry scales: 1/sqrt(d) of Pi times 1/sqrt(d) of the N(0,1)-scale centroids (grouped:
+    // 1/sqrt(32) of a Hadamard block times 1/sqrt(d_g)); prod signs: sqrt(pi/2)/d
+    const float cI = a.scale_log2 * (GRP ? 1.f / 32.f : 1.f / 128.f);
+    const float cS = GRP ? a.scale_log2 * 0.018042195912175807f
+                         : a.scale_log2 * 1.2533141373155002512f / 128.f;
+#pragma unroll
+    for (int st = 0; st < NSET; ++st) {
+      build_table<Lo::MI, PI, SL>(lutI + st * Lo::SETI, qrT, 0, st, sCen, cI, PI, threadIdx.x, NT);
+      if constexpr (PROD)
+        build_table<0, 16, SL>(lutS + st * Lo::SETS, sqT, 0, st, sCen, cS, 16, threadIdx.x, NT);
+      if constexpr (GRP)
+        build_table<Lo::MS, Lo::PS, SL>(lutS + st * Lo::SETS, qrT, 32, st, sCen + 16, cS,
+                                        Lo::IBS, threadIdx.x, NT);
+    }
+  }
+  __syncthreads();
+}
+
+// The block's partial from its NREC records [NREC][SL][kPartStride] at smem (m: the record's
+// reference maximum, l: the sum relative to it, max: its largest logit, o[128] from float 4):
+// relative to the block's largest logit M, written as the output (one split), as a
+// context-parallel record, or as a split partial; the last block of a (sequence, head group)
+// to finish then merges every split. Every thread of the block calls this.
+template <int NH, int SL, int NT, int NREC>
+__device__ __forceinline__ void decode_merge(const DecodeArgs& a, uint8_t* smem, int* sLastp,
+                                             const int16_t* gheads, int nh, int b, int split) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int& sLast = *sLastp;
+  float* sM = reinterpret_cast<float*>(smem);
+  __syncthreads();
+  if (warp < nh) {
+    // partial of this block relative to its largest logit M
+    const int h = warp, hq = gheads[h];
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NREC; ++w) M = fmaxf(M, sM[(w * SL + h) * kPartStride + 2]);
+    float Lsum = 0.f, O[4] = {0.f, 0.f, 0.f, 0.f};
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NREC; ++w) {
+        const float* src = sM + (w * SL + h) * kPartStride;
+        if (src[0] == -INFINITY) continue;
+        const float f = ex2(src[0] - M);
+        Lsum = fmaf(f, src[1], Lsum);
+        const float4 ov = *reinterpret_cast<const float4*>(src + 4 + 4 * lane);
+        O[0] = fmaf(f, ov.x, O[0]);
+        O[1] = fmaf(f, ov.y, O[1]);
+        O[2] = fmaf(f, ov.z, O[2]);
+        O[3] = fmaf(f, ov.w, O[3]);
+      }
+    }
+    const int64_t orow = (static_cast<int64_t>(b) * a.n_q_heads + hq) * kD + 4 * lane;
+    if (a.n_splits == 1 && a.part_out != nullptr) {
+      float* dst = a.part_out + (static_cast<int64_t>(b) * a.n_q_heads + hq) * kPartStride;
+      if (lane == 0) *reinterpret_cast<float4*>(dst) = make_float4(M, Lsum, 0.f, 0.f);
+      *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = make_float4(O[0], O[1], O[2], O[3]);
+    } else if (a.n_splits == 1) {
+      const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+      if (a.out_f32) {
+        *reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow) =
+            make_float4(O[0] * inv, O[1] * inv, O[2] * inv, O[3] * inv);
+      } else {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(O[0] * inv, O[1] * inv);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(O[2] * inv, O[3] * inv);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + orow) = pk;
+      }
+    } else {
+      float* dst = a.part + ((static_cast<int64_t>(b) * a.n_q_heads + hq) * a.n_splits + split) * kPartStride;
+      if (lane == 0) { dst[0] = M; dst[1] = Lsum; }
+      *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = make_float4(O[0], O[1], O[2], O[3]);
+    }
+  }
+  if (a.n_splits == 1) return;
+
+  // ---------------- the last block of this (sequence, head group) merges all splits
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int* ctr = a.counters + static_cast<int64_t>(b) * a.n_q_heads + gheads[0];
+    sLast = atomicAdd(ctr, 1) == a.n_splits - 1;
+  }
+  __syncthreads();
+  if (!sLast) return;
+  __threadfence();
+  // Every (head, split) pair's maximum and sum, then every (head, channel quad, split slice)
+  // item's weighted partial outputs, are loaded by all threads at once (one round trip each);
+  // the slices are summed in shared memory.
+  {
+    const int S = a.n_splits;
+    float* sMx = reinterpret_cast<float*>(smem);      // [head][S] split maxima
+    float* sLs = sMx + SL * 256;                      // [head][S] split sums
+    float* sF = sLs + SL * 256;                       // [head][S] weights
+    float* sHd = sF + SL * 256;  // [head] 1 / total sum, then [head] maxima and sums
+    float4* sAcc = reinterpret_cast<float4*>(sHd + 4 * SL);      // [slice][head][32]
+    const float* base = a.part + static_cast<int64_t>(b) * a.n_q_heads * S * kPartStride;
+    for (int i = threadIdx.x; i < nh * S; i += NT) {
+      const int h = i / S, sp = i - h * S;
+      const float* src = base + (static_cast<int64_t>(gheads[h]) * S + sp) * kPartStride;
+      sMx[h * 256 + sp] = __ldcg(src);
+      sLs[h * 256 + sp] = __ldcg(src + 1);
+    }
+    __syncthreads();
+    if (warp < nh) {
+      const int h = warp;
+      float mloc = -INFINITY;
+      for (int sp = lane; sp < S; sp += 32) mloc = fmaxf(mloc, sMx[h * 256 + sp]);
+      const float M = warp_max(mloc);
+      float lsum = 0.f;
+      for (int sp = lane; sp < S; sp += 32) {
+        const float ms = sMx[h * 256 + sp];
+        const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : ex2(ms - M);
+        sF[h * 256 + sp] = f;
+        lsum = fmaf(f, sLs[h * 256 + sp], lsum);
+      }
+      lsum = warp_sum(lsum);
+      if (lane == 0) {
+        sHd[h] = lsum > 0.f ? 1.f / lsum : 0.f;
+        sHd[SL + h] = M;
+        sHd[2 * SL + h] = lsum;
+      }
+    }
+    __syncthreads();
+    const int G = NT / (32 * nh);  // split slices
+    if (threadIdx.x < G * 32 * nh) {
+      const int h = threadIdx.x / (32 * G), r = threadIdx.x - h * 32 * G;
+      const int qd = r & 31, g = r >> 5;
+      const float* src = base + static_cast<int64_t>(gheads[h]) * S * kPartStride + 4 + 4 * qd;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      int sp = g;
+      for (; sp + 3 * G < S; sp += 4 * G) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = __ldcg(reinterpret_cast<const float4*>(src + static_cast<int64_t>(sp + u * G) * kPartStride));
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float f = sF[h * 256 + sp + u * G];
+          acc.x = fmaf(f, v[u].x, acc.x); acc.y = fmaf(f, v[u].y, acc.y);
+          acc.z = fmaf(f, v[u].z, acc.z); acc.w = fmaf(f, v[u].w, acc.w);
+        }
+      }
+      for (; sp < S; sp += G) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(src + static_cast<int64_t>(sp) * kPartStride));
+        const float f = sF[h * 256 + sp];
+        acc.x = fmaf(f, v.x, acc.x); acc.y = fmaf(f, v.y, acc.y);
+        acc.z = fmaf(f, v.z, acc.z); acc.w = fmaf(f, v.w, acc.w);
+      }
+      sAcc[(g * nh + h) * 32 + qd] = acc;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32 * nh) {
+      const int h = threadIdx.x >> 5, qd = threadIdx.x & 31, hq = gheads[h];
+      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int g = 0; g < G; ++g) {
+        const float4 v = sAcc[(g * nh + h) * 32 + qd];
+        O.x += v.x; O.y += v.y; O.z += v.z; O.w += v.w;
+      }
+      const float inv = sHd[h];
+      const int64_t orow = (static_cast<int64_t>(b) * a.n_q_heads + hq) * kD + 4 * qd;
+      if (a.part_out != nullptr) {
+        float* dst = a.part_out + (static_cast<int64_t>(b) * a.n_q_heads + hq) * kPartStride;
+        if (qd == 0) *reinterpret_cast<float4*>(dst) = make_float4(sHd[SL + h], sHd[2 * SL + h], 0.f, 0.f);
+        *reinterpret_cast<float4*>(dst + 4 + 4 * qd) = O;
+      } else if (a.out_f32) {
+        *reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow) =
+            make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
+      } else {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(O.x * inv, O.y * inv);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(O.z * inv, O.w * inv);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + orow) = pk;
+      }
+    }
+  }
+  if (threadIdx.x == 0) a.counters[static_cast<int64_t>(b) * a.n_q_heads + gheads[0]] = 0;
+}
+
 template <int MB, int VB, int NH, int K, int NSET>
 __global__ void __launch_bounds__(Shape<NSET>::threads, 1) k_decode(const __grid_constant__ DecodeArgs a) {
   using Lo = Lay<MB, VB, K, NSET, NH>;
@@ -330,13 +649,8 @@ __global__ void __launch_bounds__(Shape<NSET>::threads, 1) k_decode(const __grid
   static_assert(Lo::fits, "decode shared memory budget");
   constexpr bool HAS_V = VB != 0;
   extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* lutI = smem + Lo::lutI;
-  uint8_t* lutS = smem + Lo::lutS;
-  float* qrT = reinterpret_cast<float*>(smem + Lo::qrT);
-  float* sqT = reinterpret_cast<float*>(smem + Lo::sqT);
-  uint8_t* qhi = smem + Lo::qhi;
-  uint8_t* qlo = smem + Lo::qlo;
-  float* qinv = reinterpret_cast<float*>(smem + Lo::qinv);
+  const uint8_t* lutI = smem + Lo::lutI;
+  const uint8_t* lutS = smem + Lo::lutS;
   __shared__ int sLast;
   __shared__ float sCen[32];
 
@@ -382,123 +696,7 @@ __global__ void __launch_bounds__(Shape<NSET>::threads, 1) k_decode(const __grid
     }
 
     // ---------------- prologue: rotate q, project with S_rot, build the tables
-    const DevTables* __restrict__ tab = a.tab;
-    // S_rot rows [16 warp, 16 warp + 16) as mma.sync A fragments (warps 0..7)
-    uint32_t afr[8][4];
-    if (PROD && warp < 8) {
-      const int g = lane >> 2, t = lane & 3;
-      const uint32_t* r0 = reinterpret_cast<const uint32_t*>(tab->s_rot + (16 * warp + g) * kD);
-      const uint32_t* r1 = r0 + 8 * kD / 2;
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        afr[kk][0] = __ldg(r0 + kk * 8 + t);
-        afr[kk][1] = __ldg(r1 + kk * 8 + t);
-        afr[kk][2] = __ldg(r0 + kk * 8 + 4 + t);
-        afr[kk][3] = __ldg(r1 + kk * 8 + 4 + t);
-      }
-    }
-    if (warp < 8) {
-      // q_rot of head slot `warp` (zeros for empty slots): signs, then the 128-point
-      // transform with 4 values per lane (2 stages in registers, 5 across lanes)
-      float v[4] = {0.f, 0.f, 0.f, 0.f};
-      if (warp < nh) {
-        const int hq = gheads[warp];
-        const int64_t qoff = (static_cast<int64_t>(b) * a.n_q_heads + hq) * kD;
-        if constexpr (GRP) {
-          // chain order: the outlier channels, then the normal channels
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int c = tab->chan[4 * lane + i];
-            v[i] = a.q_f32 ? static_cast<const float*>(a.q)[qoff + c]
-                           : __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t*>(a.q)[qoff + c]) << 16);
-          }
-        } else {
-          if (a.q_f32) load4<true>(static_cast<const float*>(a.q) + qoff, 4 * lane, v);
-          else load4<false>(static_cast<const uint16_t*>(a.q) + qoff, 4 * lane, v);
-        }
-        const uint32_t sw = tab->sign_bits[lane >> 3];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = flip_sign(v[i], sw, (4 * lane + i) & 31);
-        // 128-point transform; grouped: 32-point blocks (lanes 8k .. 8k + 7)
-        fwht_reg<4>(v);
-#pragma unroll
-        for (int mm = 1; mm < (GRP ? 8 : 32); mm <<= 1) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float other = __shfl_xor_sync(kFull, v[i], mm);
-            v[i] = (lane & mm) ? (other - v[i]) : (v[i] + other);
-          }
-        }
-      }
-      // power-of-two scale so the fp16 hi/lo split neither overflows nor underflows
-      float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
-      amax = warp_max(amax);
-      const uint32_t ex = (__float_as_uint(amax) >> 23) & 0xffu;
-      const bool big = ex >= 12u;
-      const float scl = big ? __uint_as_float((264u - ex) << 23) : 1.f;
-      const float inv = big ? __uint_as_float((ex - 10u) << 23) : 1.f;
-      if (lane == 0) qinv[warp] = inv;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int j = 4 * lane + i;
-        if (warp < SL) qrT[j * SL + warp] = v[i];
-        const float sv = v[i] * scl;
-        const __half hi = __float2half_rn(sv);
-        const __half lo = __float2half_rn(sv - __half2float(hi));
-        reinterpret_cast<__half*>(qhi + warp * kQStride)[j] = hi;
-        reinterpret_cast<__half*>(qlo + warp * kQStride)[j] = lo;
-      }
-    }
-    if (threadIdx.x < 32) sCen[threadIdx.x] = (&tab->cent[0][0])[threadIdx.x];
-    __syncthreads();
-    if (PROD && warp < 8) {
-      // Sq = S_rot q_rot / sqrt(d) for the head slots on tensor cores: mma.sync m16n8k16
-      // (fp16 S_rot is exact; q_rot enters as hi + lo fp16 halves; fp32 accumulation).
-      const int g = lane >> 2, t = lane & 3;
-      float c0 = 0.f, c1 = 0.f, c2 = 0.f, c3 = 0.f;
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const int k0 = 16 * kk;
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          const uint8_t* bq = (part ? qlo : qhi) + g * kQStride;
-          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(bq + (k0 + 2 * t) * 2);
-          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(bq + (k0 + 8 + 2 * t) * 2);
-          asm volatile(
-              "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
-              "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};\n"
-              : "+f"(c0), "+f"(c1), "+f"(c2), "+f"(c3)
-              : "r"(afr[kk][0]), "r"(afr[kk][1]), "r"(afr[kk][2]), "r"(afr[kk][3]), "r"(b0), "r"(b1));
-        }
-      }
-      if (2 * t < SL) {  // columns 2t, 2t + 1 are head slots
-        const float s0 = qinv[2 * t] * 0.088388347648318440550f;      // / sqrt(128)
-        const float s1 = qinv[2 * t + 1] * 0.088388347648318440550f;
-        const int j0 = 16 * warp + g;
-        sqT[j0 * SL + 2 * t] = c0 * s0;
-        sqT[j0 * SL + 2 * t + 1] = c1 * s1;
-        sqT[(j0 + 8) * SL + 2 * t] = c2 * s0;
-        sqT[(j0 + 8) * SL + 2 * t + 1] = c3 * s1;
-      }
-    }
-    if constexpr (PROD) __syncthreads();
-    {
-      // entry scales: 1/sqrt(d) of Pi times 1/sqrt(d) of the N(0,1)-scale centroids (grouped:
-      // 1/sqrt(32) of a Hadamard block times 1/sqrt(d_g)); prod signs: sqrt(pi/2)/d
-      const float cI = a.scale_log2 * (GRP ? 1.f / 32.f : 1.f / 128.f);
-      const float cS = GRP ? a.scale_log2 * 0.018042195912175807f
-                           : a.scale_log2 * 1.2533141373155002512f / 128.f;
-#pragma unroll
-      for (int st = 0; st < NSET; ++st) {
-        build_table<Lo::MI, PI, SL>(lutI + st * Lo::SETI, qrT, 0, st, sCen, cI, PI, threadIdx.x, NT);
-        if constexpr (PROD)
-          build_table<0, 16, SL>(lutS + st * Lo::SETS, sqT, 0, st, sCen, cS, 16, threadIdx.x, NT);
-        if constexpr (GRP)
-          build_table<Lo::MS, Lo::PS, SL>(lutS + st * Lo::SETS, qrT, 32, st, sCen + 16, cS,
-                                          Lo::IBS, threadIdx.x, NT);
-      }
-    }
-    __syncthreads();
+    decode_prologue<Lo, K, NSET, NT>(a, smem, sCen, gheads, nh, b);
     grid_dependency_wait();
     t1 = min(a.len[b], t0 + a.tokens_per_split);
 
@@ -741,156 +939,7 @@ __global__ void __launch_bounds__(Shape<NSET>::threads, 1) k_decode(const __grid
       }
     }
   }
-  __syncthreads();
-  if (warp < nh) {
-    // partial of this block relative to its largest logit M
-    const int h = warp, hq = gheads[h];
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < NWp; ++w) M = fmaxf(M, sM[(w * SL + h) * kPartStride + 2]);
-    float Lsum = 0.f, O[4] = {0.f, 0.f, 0.f, 0.f};
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < NWp; ++w) {
-        const float* src = sM + (w * SL + h) * kPartStride;
-        if (src[0] == -INFINITY) continue;
-        const float f = ex2(src[0] - M);
-        Lsum = fmaf(f, src[1], Lsum);
-        const float4 ov = *reinterpret_cast<const float4*>(src + 4 + 4 * lane);
-        O[0] = fmaf(f, ov.x, O[0]);
-        O[1] = fmaf(f, ov.y, O[1]);
-        O[2] = fmaf(f, ov.z, O[2]);
-        O[3] = fmaf(f, ov.w, O[3]);
-      }
-    }
-    const int64_t orow = (static_cast<int64_t>(b) * a.n_q_heads + hq) * kD + 4 * lane;
-    if (a.n_splits == 1 && a.part_out != nullptr) {
-      float* dst = a.part_out + (static_cast<int64_t>(b) * a.n_q_heads + hq) * kPartStride;
-      if (lane == 0) *reinterpret_cast<float4*>(dst) = make_float4(M, Lsum, 0.f, 0.f);
-      *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = make_float4(O[0], O[1], O[2], O[3]);
-    } else if (a.n_splits == 1) {
-      const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-      if (a.out_f32) {
-        *reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow) =
-            make_float4(O[0] * inv, O[1] * inv, O[2] * inv, O[3] * inv);
-      } else {
-        __nv_bfloat162 lo = __floats2bfloat162_rn(O[0] * inv, O[1] * inv);
-        __nv_bfloat162 hi = __floats2bfloat162_rn(O[2] * inv, O[3] * inv);
-        uint2 pk;
-        pk.x = *reinterpret_cast<uint32_t*>(&lo);
-        pk.y = *reinterpret_cast<uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + orow) = pk;
-      }
-    } else {
-      float* dst = a.part + ((static_cast<int64_t>(b) * a.n_q_heads + hq) * a.n_splits + split) * kPartStride;
-      if (lane == 0) { dst[0] = M; dst[1] = Lsum; }
-      *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = make_float4(O[0], O[1], O[2], O[3]);
-    }
-  }
-  if (a.n_splits == 1) return;
-
-  // ---------------- the last block of this (sequence, head group) merges all splits
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int* ctr = a.counters + static_cast<int64_t>(b) * a.n_q_heads + gheads[0];
-    sLast = atomicAdd(ctr, 1) == a.n_splits - 1;
-  }
-  __syncthreads();
-  if (!sLast) return;
-  __threadfence();
-  // Every (head, split) pair's maximum and sum, then every (head, channel quad, split slice)
-  // item's weighted partial outputs, are loaded by all threads at once (one round trip each);
-  // the slices are summed in shared memory.
-  {
-    const int S = a.n_splits;
-    float* sMx = reinterpret_cast<float*>(smem);      // [head][S] split maxima
-    float* sLs = sMx + SL * 256;                      // [head][S] split sums
-    float* sF = sLs + SL * 256;                       // [head][S] weights
-    float* sHd = sF + SL * 256;  // [head] 1 / total sum, then [head] maxima and sums
-    float4* sAcc = reinterpret_cast<float4*>(sHd + 4 * SL);      // [slice][head][32]
-    const float* base = a.part + static_cast<int64_t>(b) * a.n_q_heads * S * kPartStride;
-    for (int i = threadIdx.x; i < nh * S; i += NT) {
-      const int h = i / S, sp = i - h * S;
-      const float* src = base + (static_cast<int64_t>(gheads[h]) * S + sp) * kPartStride;
-      sMx[h * 256 + sp] = __ldcg(src);
-      sLs[h * 256 + sp] = __ldcg(src + 1);
-    }
-    __syncthreads();
-    if (warp < nh) {
-      const int h = warp;
-      float mloc = -INFINITY;
-      for (int sp = lane; sp < S; sp += 32) mloc = fmaxf(mloc, sMx[h * 256 + sp]);
-      const float M = warp_max(mloc);
-      float lsum = 0.f;
-      for (int sp = lane; sp < S; sp += 32) {
-        const float ms = sMx[h * 256 + sp];
-        const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : ex2(ms - M);
-        sF[h * 256 + sp] = f;
-        lsum = fmaf(f, sLs[h * 256 + sp], lsum);
-      }
-      lsum = warp_sum(lsum);
-      if (lane == 0) {
-        sHd[h] = lsum > 0.f ? 1.f / lsum : 0.f;
-        sHd[SL + h] = M;
-        sHd[2 * SL + h] = lsum;
-      }
-    }
-    __syncthreads();
-    const int G = NT / (32 * nh);  // split slices
-    if (threadIdx.x < G * 32 * nh) {
-      const int h = threadIdx.x / (32 * G), r = threadIdx.x - h * 32 * G;
-      const int qd = r & 31, g = r >> 5;
-      const float* src = base + static_cast<int64_t>(gheads[h]) * S * kPartStride + 4 + 4 * qd;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      int sp = g;
-      for (; sp + 3 * G < S; sp += 4 * G) {
-        float4 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) v[u] = __ldcg(reinterpret_cast<const float4*>(src + static_cast<int64_t>(sp + u * G) * kPartStride));
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float f = sF[h * 256 + sp + u * G];
-          acc.x = fmaf(f, v[u].x, acc.x); acc.y = fmaf(f, v[u].y, acc.y);
-          acc.z = fmaf(f, v[u].z, acc.z); acc.w = fmaf(f, v[u].w, acc.w);
-        }
-      }
-      for (; sp < S; sp += G) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(src + static_cast<int64_t>(sp) * kPartStride));
-        const float f = sF[h * 256 + sp];
-        acc.x = fmaf(f, v.x, acc.x); acc.y = fmaf(f, v.y, acc.y);
-        acc.z = fmaf(f, v.z, acc.z); acc.w = fmaf(f, v.w, acc.w);
-      }
-      sAcc[(g * nh + h) * 32 + qd] = acc;
-    }
-    __syncthreads();
-    if (threadIdx.x < 32 * nh) {
-      const int h = threadIdx.x >> 5, qd = threadIdx.x & 31, hq = gheads[h];
-      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int g = 0; g < G; ++g) {
-        const float4 v = sAcc[(g * nh + h) * 32 + qd];
-        O.x += v.x; O.y += v.y; O.z += v.z; O.w += v.w;
-      }
-      const float inv = sHd[h];
-      const int64_t orow = (static_cast<int64_t>(b) * a.n_q_heads + hq) * kD + 4 * qd;
-      if (a.part_out != nullptr) {
-        float* dst = a.part_out + (static_cast<int64_t>(b) * a.n_q_heads + hq) * kPartStride;
-        if (qd == 0) *reinterpret_cast<float4*>(dst) = make_float4(sHd[SL + h], sHd[2 * SL + h], 0.f, 0.f);
-        *reinterpret_cast<float4*>(dst + 4 + 4 * qd) = O;
-      } else if (a.out_f32) {
-        *reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow) =
-            make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
-      } else {
-        __nv_bfloat162 lo = __floats2bfloat162_rn(O.x * inv, O.y * inv);
-        __nv_bfloat162 hi = __floats2bfloat162_rn(O.z * inv, O.w * inv);
-        uint2 pk;
-        pk.x = *reinterpret_cast<uint32_t*>(&lo);
-        pk.y = *reinterpret_cast<uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + orow) = pk;
-      }
-    }
-  }
-  if (threadIdx.x == 0) a.counters[static_cast<int64_t>(b) * a.n_q_heads + gheads[0]] = 0;
+  decode_merge<NH, SL, NT, NWp>(a, smem, &sLast, gheads, nh, b, split);
 }
 
 // Launch one instantiation (dynamic shared memory configured on first use; programmatic
@@ -919,6 +968,8 @@ tq_status run_decode(const DecodeArgs& a, dim3 grid, bool pdl, cudaStream_t st) 
   if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return TQ_ECUDA;
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ECUDA;
 }
+
+
 
 // Two table sets where the layout fits the shared memory (and never for grouped keys, whose
 // two segments already take two table kinds).

@@ -902,6 +902,19 @@ tq_status launch_selftest_wait(uint32_t limit_us, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ECUDA;
 }
 
+int* device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  static int* addr[64] = {};
+  if (addr[dev] == nullptr) {
+    int* p = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_tq_device_error) != cudaSuccess)
+      return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
 tq_status take_device_error(cudaStream_t st) {
   if (cudaStreamSynchronize(st) != cudaSuccess) return TQ_ECUDA;
   int v = 0;

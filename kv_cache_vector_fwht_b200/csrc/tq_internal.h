@@ -89,6 +89,9 @@ tq_status launch_dequantize_keys(const tq_quantizer* q, tq_key_planes planes, in
 bool keys_tc_ok(const tq_quantizer* q, int dtype);
 tq_status launch_keys_tc(const tq_quantizer* q, const void* x, int64_t n_rows, int64_t ld,
                          tq_key_planes out, RowMap map, cudaStream_t st);
+// Device address of the error word that kernels set when a bounded wait runs out (the current
+// device; nullptr if it cannot be looked up).
+int* device_error_word();
 // Synchronise `st`; TQ_ETIMEOUT (and clear the flag) if a kernel gave up a bounded wait.
 tq_status take_device_error(cudaStream_t st);
 // A one-thread kernel whose bounded mbarrier wait runs out (sets the error flag).
