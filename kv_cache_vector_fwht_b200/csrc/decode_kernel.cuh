@@ -319,24 +319,6 @@ __device__ __forceinline__ void build_table(uint8_t* lut, const float* x, int c0
 // K = kMse: s = n16 <Pi q, c[idx]>; kProd: + r16 sqrt(pi/2)/d <S q, 2 sigma - 1>;
 // kGrp: s = n_o <Pi_o q_o, c_o[idx_o]> + n_n <Pi_n q_n, c_n[idx_n]> over the two channel
 // groups (Pi_g: 32-point Hadamard blocks after the group's signs).
-// L2 prefetch of the packed rows of one 32-token chunk starting at ts (tokens below tp1):
-// the index, sign, norm, value-code and value-parameter planes, one 128-byte line a lane.
-template <int IB, int NB, int VQB, bool PROD, bool HAS_V>
-__device__ __forceinline__ void prefetch_rows(const DecodeArgs& a, int64_t kvrow, int ts, int tp1,
-                                              int lane) {
-  const int n = min(32, tp1 - ts);
-  if (n <= 0) return;
-  const uint8_t* rng[5] = {a.k_idx + (kvrow + ts) * IB, a.k_sgn + (kvrow + ts) * 16,
-                           reinterpret_cast<const uint8_t*>(a.k_nrm) + (kvrow + ts) * NB,
-                           a.v_q + (kvrow + ts) * VQB,
-                           reinterpret_cast<const uint8_t*>(a.v_par) + (kvrow + ts) * 16};
-  const int len_b[5] = {n * IB, PROD ? n * 16 : 0, n * NB, HAS_V ? n * VQB : 0, HAS_V ? n * 16 : 0};
-#pragma unroll
-  for (int r = 0; r < 5; ++r)
-    for (int o = lane * 128; o < len_b[r]; o += 32 * 128)
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(rng[r] + o));
-}
-
 // The query prologue of a block (it reads only the query and the quantizer's tables): q_rot =
 // H (s . q) per head slot (grouped: gathered in channel order, 32-point blocks), Sq = S_rot
 // q_rot / sqrt(d) on tensor cores (mma.sync, fp16 hi + lo halves of q_rot, fp32 accumulation),
