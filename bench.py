@@ -56,7 +56,8 @@ QUANT_MODES = [("mse", 1), ("mse", 2), ("mse", 3), ("mse", 4), ("prod", 2), ("pr
                ("prod", 4), ("grouped", 1), ("grouped", 2), ("grouped", 3)]
 # kernel launches of one tq_append_decode step: the fused append and the fused decode
 LAUNCHES_PER_STEP = 2
-DECODE_SOURCES = ["decode.cu", "tq_device.cuh", "tq_internal.h"]
+DECODE_SOURCES = ["decode_kernel.cuh", "decode.cu", "decode_prod.cu", "decode_mse.cu",
+                  "decode_grp.cu", "tq_device.cuh", "tq_internal.h"]
 
 
 def key_bytes(bits):      # prod mode: (bits - 1)-bit indices (3-bit stored in 4) + signs + norms
@@ -98,6 +99,9 @@ def parse(argv=None):
                     help="with --only quantize: one mode and width, or all")
     ap.add_argument("--extra-steps", type=int, default=200,
                     help="timed steps of each non-headline decode workload")
+    ap.add_argument("--key-only", action="store_true",
+                    help="with --only decode: a key-only cache decoded without outputs (the "
+                         "table lookups alone)")
     return ap.parse_args(argv)
 
 
@@ -247,7 +251,7 @@ class DecodeBench:
     """A decode workload on the device: the prefilled packed cache, fresh tokens and queries
     for every step, the decode workspace and the L2 flush buffer."""
 
-    def __init__(self, tq, torch, dev, name: str, n_steps: int, rank: int):
+    def __init__(self, tq, torch, dev, name: str, n_steps: int, rank: int, key_only=False):
         wl = DECODE_WORKLOADS[name]
         self.name, self.wl, self.tq, self.torch, self.dev = name, wl, tq, torch, dev
         B, Hq, Hkv, N = wl["batch"], wl["n_q_heads"], wl["n_kv_heads"], wl["ctx"]
@@ -276,11 +280,13 @@ class DecodeBench:
         K = K.to(torch.bfloat16)
         self.qz = tq.tq_build_codebook(128, wl["key_bits"], "prod", wl["qseed"])
         cap = ((N + extra + 15) // 16) * 16
-        self.cache = tq.KVCache(self.qz, B, Hkv, cap, value_bits=wl["value_bits"], device=dev)
-        tq.tq_append(self.qz, self.cache, K.contiguous(), V.contiguous())   # prefill (untimed)
+        self.key_only = key_only
+        vb = 0 if key_only else wl["value_bits"]
+        self.cache = tq.KVCache(self.qz, B, Hkv, cap, value_bits=vb, device=dev)
+        tq.tq_append(self.qz, self.cache, K.contiguous(), None if key_only else V.contiguous())
         del K, V
         self.ws = tq.alloc_decode_workspace(self.cache, Hq, dev)
-        self.out = torch.empty((B, Hq, 128), device=dev, dtype=torch.bfloat16)
+        self.out = None if key_only else torch.empty((B, Hq, 128), device=dev, dtype=torch.bfloat16)
         self.flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
         self.i = 0
 
@@ -288,14 +294,19 @@ class DecodeBench:
         """One decode step through the public API: append this step's token per KV head,
         then decode (one tq_append_decode call)."""
         i = self.i
-        self.tq.tq_append_decode(self.qz, self.cache, self.Kn[i], self.Vn[i], self.Qs[i],
-                                 self.out, self.ws)
+        if self.key_only:   # the decode's table lookups alone (no values, no outputs)
+            self.tq.tq_decode_attention(self.qz, self.cache, self.Qs[i], None, self.ws)
+        else:
+            self.tq.tq_append_decode(self.qz, self.cache, self.Kn[i], self.Vn[i], self.Qs[i],
+                                     self.out, self.ws)
         self.i += 1
 
     def bytes_per_step(self, mean_len: float) -> float:
         """Algorithmic HBM bytes of one step: the cache read by the decode, the appended rows
         (bf16 in, packed out), the query and the output."""
         wl = self.wl
+        if self.key_only:   # keys read, the query; no append, no values, no output
+            return self.B * self.Hkv * mean_len * key_bytes(wl["key_bits"]) + self.B * self.Hq * 256
         per = key_bytes(wl["key_bits"]) + value_bytes(wl["value_bits"])
         return (self.B * self.Hkv * mean_len * per
                 + self.B * self.Hkv * (2 * 256 + per)
@@ -509,7 +520,8 @@ def run_tq(args):
             print(json.dumps({"key_quantize": r}))
         return _finish(world)
     if args.only == "decode":
-        d = DecodeBench(tq, torch, dev, args.decode_workload, warm + steps, rank)
+        d = DecodeBench(tq, torch, dev, args.decode_workload, warm + steps, rank,
+                        key_only=args.key_only)
         r = d.run(steps, warm, world)
         if rank == 0:
             print(json.dumps({args.decode_workload: r}))

@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(256) k_keys_full(KeyArgs a) {
 
   extern __shared__ __align__(16) float smem[];
   float* sST = smem;                          // prod: S_rot^T in fp32, [i][j] = S_rot[j][i]
-  float* sRho = smem + (PROD ? kD * kD : 0);  // prod: [8 warps][16 rows][kRhoStride]
+  float* sRho = smem + (PROD ? kD * kD : 0);  // prod: [warps][16 rows][kRhoStride]
 
   const DevTables* __restrict__ tab = a.tab;
   float thr[NL - 1], cen[NL];
@@ -75,12 +75,13 @@ __global__ void __launch_bounds__(256) k_keys_full(KeyArgs a) {
   }
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = static_cast<int>(blockDim.x >> 5);
   const int hf = lane & 1, rl = lane >> 1;
   const uint32_t hmask = static_cast<uint32_t>(hf) << 31;
   const int64_t n_groups = (a.n_rows + 15) / 16;
 
-  for (int64_t g = static_cast<int64_t>(blockIdx.x) * 8 + warp; g < n_groups;
-       g += static_cast<int64_t>(gridDim.x) * 8) {
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * nwarps + warp; g < n_groups;
+       g += static_cast<int64_t>(gridDim.x) * nwarps) {
     const int64_t row = g * 16 + rl;
     const bool valid = row < a.n_rows;
     const int64_t src = valid ? row : a.n_rows - 1;
@@ -378,15 +379,23 @@ int grid_for(K kernel, int block, size_t smem, int64_t work_items_per_block, int
 template <int MODE, int BITS, bool F32>
 tq_status run_full(const KeyArgs& a, cudaStream_t st) {
   constexpr bool PROD = MODE == TQ_MODE_PROD;
-  const size_t smem = PROD ? (kD * kD + 8 * 16 * kRhoStride) * sizeof(float) : 0;
+  // 8 warps (128 rows) per block; inputs too small to give every SM a block take 2-warp
+  // blocks (32 rows each, 4x the blocks)
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int warps = a.n_rows < static_cast<int64_t>(sm_count(dev)) * 128 ? 2 : 8;
+  const size_t smem = PROD ? (kD * kD + warps * 16 * kRhoStride) * sizeof(float) : 0;
   auto kern = k_keys_full<MODE, BITS, F32>;
-  if (smem > 48 * 1024) {
+  static bool attr_set = false;
+  if (PROD && !attr_set) {
+    const size_t smem_max = (kD * kD + 8 * 16 * kRhoStride) * sizeof(float);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
+                             static_cast<int>(smem_max)) != cudaSuccess)
       return TQ_ECUDA;
+    attr_set = true;
   }
-  const int grid = grid_for(kern, 256, smem, 8 * 16, a.n_rows);
-  kern<<<grid, 256, smem, st>>>(a);
+  const int grid = grid_for(kern, 32 * warps, smem, warps * 16, a.n_rows);
+  kern<<<grid, 32 * warps, smem, st>>>(a);
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ECUDA;
 }
 
