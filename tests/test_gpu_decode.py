@@ -347,8 +347,8 @@ def two_sets():
 ])
 def test_decode_eight_heads_per_cta(mode, bits, vbits, hq, hm, decode_shape):
     """More than 4 query heads per KV head, in both block shapes: one block serving up to 8
-    of them with two table sets (12 warps, nibble sign tables for prod, one token per P.V
-    step), and blocks of at most 4."""
+    of them with two table sets (8 warps, byte tables for both lookup segments, P.V over
+    every head of the block), and blocks of at most 4 (one set, 16 warps)."""
     require_cuda()
     qo, qg, oc, cache, Q = small_case(150 + bits + hq, 2, hq, 2, [1000, 613], 1024, bits, vbits, mode)
     out, sc, _ = run_decode(qg, cache, Q, torch.bfloat16, torch.float32, head_map=hm,
