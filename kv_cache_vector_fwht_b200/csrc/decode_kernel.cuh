@@ -166,6 +166,11 @@ __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
 }
 
+// L2 prefetch of [p, p + bytes) by the TMA unit (p 16-byte aligned, bytes a multiple of 16)
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -259,15 +264,25 @@ __device__ __forceinline__ void segment_lookups(uint64_t (&acc)[NS][2], const ui
   }
 }
 
+// Float index of (coordinate j, head slot s) in a [128][SL] query array whose 16-byte units
+// (4 head slots of one coordinate) are XOR-permuted by (j / XC) & 7 within aligned groups of
+// 8 units: the table builders' lanes take consecutive byte positions p and read coordinate
+// XC p + f at the same f, which lands them in 8 different bank groups per 128-byte phase.
+template <int XC, int SL>
+__device__ __forceinline__ int xidx(int j, int s) {
+  const int u = j * (SL / 4) + (s >> 2);
+  return 4 * (u ^ ((j / XC) & 7)) + (s & 3);
+}
+
 // Build the lookup table of one segment for table set st: NPOS positions of bytes whose
 // coordinates c0 + CPB p + f (f < CPB coordinates per byte) carry CB-bit codes (CB = 0: QJL
 // sign bits, value +-cs); entry e = sum_f x[coordinate][head] * cen[code_f(e)] * cs for the
 // canonical bytes (top bit clear; 3-bit nibble bytes: high code below 4). x is a [128][SL]
-// f32 array (q_rot or Sq), 4 heads from column 4 st. An item (position, high nibble) loads
+// f32 array (q_rot or Sq; laid out by xidx<XC, SL>), 4 heads from column 4 st. An item (position, high nibble) loads
 // its coordinates once, sums the high nibble's coordinates once and writes the entries of
 // every low nibble, whose codes are compile-time constants (centroids from registers).
 // Positions p >= nvalid are padding of the grouped normal segment and stay zero.
-template <int CB, int NPOS, int SL>
+template <int CB, int NPOS, int SL, int XC>
 __device__ __forceinline__ void build_table(uint8_t* lut, const float* x, int c0, int st,
                                             const float* cen, float cs, int nvalid, int tid,
                                             int nthreads) {
@@ -287,7 +302,7 @@ __device__ __forceinline__ void build_table(uint8_t* lut, const float* x, int c0
     float4 xs[CPB];
 #pragma unroll
     for (int f = 0; f < CPB; ++f)
-      xs[f] = ok ? *reinterpret_cast<const float4*>(x + (c0 + CPB * p + f) * SL + 4 * st)
+      xs[f] = ok ? *reinterpret_cast<const float4*>(x + xidx<XC, SL>(c0 + CPB * p + f, 4 * st))
                  : make_float4(0.f, 0.f, 0.f, 0.f);
     float4 ph = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -329,6 +344,8 @@ __device__ __forceinline__ void decode_prologue(const DecodeArgs& a, uint8_t* sm
                                                 const int16_t* gheads, int nh, int b) {
   constexpr int SL = Lo::SL, PI = Lo::PI;
   constexpr bool PROD = K == kProd, GRP = K == kGrp;
+  // coordinates per index byte: the swizzle key of q_rot (the sign tables read Sq by 8)
+  constexpr int XCI = 8 / storage_width_c(Lo::MI);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint8_t* lutI = smem + Lo::lutI;
   uint8_t* lutS = smem + Lo::lutS;
@@ -396,7 +413,7 @@ __device__ __forceinline__ void decode_prologue(const DecodeArgs& a, uint8_t* sm
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int j = 4 * lane + i;
-      if (warp < SL) qrT[j * SL + warp] = v[i];
+      if (warp < SL) qrT[xidx<XCI, SL>(j, warp)] = v[i];
       const float sv = v[i] * scl;
       const __half hi = __float2half_rn(sv);
       const __half lo = __float2half_rn(sv - __half2float(hi));
@@ -430,10 +447,10 @@ __device__ __forceinline__ void decode_prologue(const DecodeArgs& a, uint8_t* sm
       const float s0 = qinv[2 * t] * 0.088388347648318440550f;      // / sqrt(128)
       const float s1 = qinv[2 * t + 1] * 0.088388347648318440550f;
       const int j0 = 16 * warp + g;
-      sqT[j0 * SL + 2 * t] = c0 * s0;
-      sqT[j0 * SL + 2 * t + 1] = c1 * s1;
-      sqT[(j0 + 8) * SL + 2 * t] = c2 * s0;
-      sqT[(j0 + 8) * SL + 2 * t + 1] = c3 * s1;
+      sqT[xidx<8, SL>(j0, 2 * t)] = c0 * s0;
+      sqT[xidx<8, SL>(j0, 2 * t + 1)] = c1 * s1;
+      sqT[xidx<8, SL>(j0 + 8, 2 * t)] = c2 * s0;
+      sqT[xidx<8, SL>(j0 + 8, 2 * t + 1)] = c3 * s1;
     }
   }
   if constexpr (PROD) __syncthreads();
@@ -445,11 +462,11 @@ __device__ __forceinline__ void decode_prologue(const DecodeArgs& a, uint8_t* sm
                          : a.scale_log2 * 1.2533141373155002512f / 128.f;
 #pragma unroll
     for (int st = 0; st < NSET; ++st) {
-      build_table<Lo::MI, PI, SL>(lutI + st * Lo::SETI, qrT, 0, st, sCen, cI, PI, threadIdx.x, NT);
+      build_table<Lo::MI, PI, SL, XCI>(lutI + st * Lo::SETI, qrT, 0, st, sCen, cI, PI, threadIdx.x, NT);
       if constexpr (PROD)
-        build_table<0, 16, SL>(lutS + st * Lo::SETS, sqT, 0, st, sCen, cS, 16, threadIdx.x, NT);
+        build_table<0, 16, SL, 8>(lutS + st * Lo::SETS, sqT, 0, st, sCen, cS, 16, threadIdx.x, NT);
       if constexpr (GRP)
-        build_table<Lo::MS, Lo::PS, SL>(lutS + st * Lo::SETS, qrT, 32, st, sCen + 16, cS,
+        build_table<Lo::MS, Lo::PS, SL, XCI>(lutS + st * Lo::SETS, qrT, 32, st, sCen + 16, cS,
                                         Lo::IBS, threadIdx.x, NT);
     }
   }
@@ -516,92 +533,90 @@ __device__ __forceinline__ void decode_merge(const DecodeArgs& a, uint8_t* smem,
   if (a.n_splits == 1) return;
 
   // ---------------- the last block of this (sequence, head group) merges all splits
-  __threadfence();
+  // One thread releases the block's partials (ordered before it by the barrier) and counts
+  // the block; the last block's thread acquires the other blocks' partials before the
+  // barrier that releases its readers.
   __syncthreads();
   if (threadIdx.x == 0) {
+    __threadfence();
     int* ctr = a.counters + static_cast<int64_t>(b) * a.n_q_heads + gheads[0];
-    sLast = atomicAdd(ctr, 1) == a.n_splits - 1;
+    const bool last = atomicAdd(ctr, 1) == a.n_splits - 1;
+    if (last) __threadfence();
+    sLast = last;
   }
   __syncthreads();
   if (!sLast) return;
-  __threadfence();
-  // Every (head, split) pair's maximum and sum, then every (head, channel quad, split slice)
-  // item's weighted partial outputs, are loaded by all threads at once (one round trip each);
-  // the slices are summed in shared memory.
+  // Item (head, channel quad, split slice) loads the (maximum, sum, output quad) records of
+  // its splits in one round trip (batches of 8) and merges them relative to their largest
+  // maximum; the slices are then merged in shared memory.
   {
     const int S = a.n_splits;
-    float* sMx = reinterpret_cast<float*>(smem);      // [head][S] split maxima
-    float* sLs = sMx + SL * 256;                      // [head][S] split sums
-    float* sF = sLs + SL * 256;                       // [head][S] weights
-    float* sHd = sF + SL * 256;  // [head] 1 / total sum, then [head] maxima and sums
-    float4* sAcc = reinterpret_cast<float4*>(sHd + 4 * SL);      // [slice][head][32]
-    const float* base = a.part + static_cast<int64_t>(b) * a.n_q_heads * S * kPartStride;
-    for (int i = threadIdx.x; i < nh * S; i += NT) {
-      const int h = i / S, sp = i - h * S;
-      const float* src = base + (static_cast<int64_t>(gheads[h]) * S + sp) * kPartStride;
-      sMx[h * 256 + sp] = __ldcg(src);
-      sLs[h * 256 + sp] = __ldcg(src + 1);
-    }
-    __syncthreads();
-    if (warp < nh) {
-      const int h = warp;
-      float mloc = -INFINITY;
-      for (int sp = lane; sp < S; sp += 32) mloc = fmaxf(mloc, sMx[h * 256 + sp]);
-      const float M = warp_max(mloc);
-      float lsum = 0.f;
-      for (int sp = lane; sp < S; sp += 32) {
-        const float ms = sMx[h * 256 + sp];
-        const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : ex2(ms - M);
-        sF[h * 256 + sp] = f;
-        lsum = fmaf(f, sLs[h * 256 + sp], lsum);
-      }
-      lsum = warp_sum(lsum);
-      if (lane == 0) {
-        sHd[h] = lsum > 0.f ? 1.f / lsum : 0.f;
-        sHd[SL + h] = M;
-        sHd[2 * SL + h] = lsum;
-      }
-    }
-    __syncthreads();
     const int G = NT / (32 * nh);  // split slices
+    float2* sML = reinterpret_cast<float2*>(smem);                  // [slice][head] (M, L)
+    float4* sAcc = reinterpret_cast<float4*>(smem + 16 * 8 * SL);   // [slice][head][32]
+    const float* base = a.part + static_cast<int64_t>(b) * a.n_q_heads * S * kPartStride;
     if (threadIdx.x < G * 32 * nh) {
       const int h = threadIdx.x / (32 * G), r = threadIdx.x - h * 32 * G;
       const int qd = r & 31, g = r >> 5;
-      const float* src = base + static_cast<int64_t>(gheads[h]) * S * kPartStride + 4 + 4 * qd;
+      const float* src = base + static_cast<int64_t>(gheads[h]) * S * kPartStride;
+      float M = -INFINITY, L = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      int sp = g;
-      for (; sp + 3 * G < S; sp += 4 * G) {
-        float4 v[4];
+      for (int sp0 = g; sp0 < S; sp0 += 8 * G) {
+        float2 ml[8];
+        float4 v[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) v[u] = __ldcg(reinterpret_cast<const float4*>(src + static_cast<int64_t>(sp + u * G) * kPartStride));
+        for (int u = 0; u < 8; ++u) {
+          const int sp = sp0 + u * G;
+          if (sp < S) {
+            const float* rec = src + static_cast<int64_t>(sp) * kPartStride;
+            ml[u] = __ldcg(reinterpret_cast<const float2*>(rec));
+            v[u] = __ldcg(reinterpret_cast<const float4*>(rec + 4 + 4 * qd));
+          } else {
+            ml[u] = make_float2(-INFINITY, 0.f);
+            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+        float mb = M;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float f = sF[h * 256 + sp + u * G];
+        for (int u = 0; u < 8; ++u) mb = fmaxf(mb, ml[u].x);
+        if (mb == -INFINITY) continue;  // no token so far
+        const float al = ex2(M - mb);   // 0 while M = -inf
+        L *= al;
+        acc.x *= al; acc.y *= al; acc.z *= al; acc.w *= al;
+        M = mb;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float f = ex2(ml[u].x - M);  // 0 for an empty split (m = -inf)
+          L = fmaf(f, ml[u].y, L);
           acc.x = fmaf(f, v[u].x, acc.x); acc.y = fmaf(f, v[u].y, acc.y);
           acc.z = fmaf(f, v[u].z, acc.z); acc.w = fmaf(f, v[u].w, acc.w);
         }
       }
-      for (; sp < S; sp += G) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(src + static_cast<int64_t>(sp) * kPartStride));
-        const float f = sF[h * 256 + sp];
-        acc.x = fmaf(f, v.x, acc.x); acc.y = fmaf(f, v.y, acc.y);
-        acc.z = fmaf(f, v.z, acc.z); acc.w = fmaf(f, v.w, acc.w);
-      }
-      sAcc[(g * nh + h) * 32 + qd] = acc;
+      if (qd == 0) sML[g * SL + h] = make_float2(M, L);
+      sAcc[(g * SL + h) * 32 + qd] = acc;
     }
     __syncthreads();
     if (threadIdx.x < 32 * nh) {
       const int h = threadIdx.x >> 5, qd = threadIdx.x & 31, hq = gheads[h];
+      float Mt = -INFINITY;
+      for (int g = 0; g < G; ++g) Mt = fmaxf(Mt, sML[g * SL + h].x);
+      float Lt = 0.f;
       float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int g = 0; g < G; ++g) {
-        const float4 v = sAcc[(g * nh + h) * 32 + qd];
-        O.x += v.x; O.y += v.y; O.z += v.z; O.w += v.w;
+      if (Mt != -INFINITY) {
+        for (int g = 0; g < G; ++g) {
+          const float2 ml = sML[g * SL + h];
+          const float f = ex2(ml.x - Mt);
+          const float4 v = sAcc[(g * SL + h) * 32 + qd];
+          Lt = fmaf(f, ml.y, Lt);
+          O.x = fmaf(f, v.x, O.x); O.y = fmaf(f, v.y, O.y);
+          O.z = fmaf(f, v.z, O.z); O.w = fmaf(f, v.w, O.w);
+        }
       }
-      const float inv = sHd[h];
+      const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
       const int64_t orow = (static_cast<int64_t>(b) * a.n_q_heads + hq) * kD + 4 * qd;
       if (a.part_out != nullptr) {
         float* dst = a.part_out + (static_cast<int64_t>(b) * a.n_q_heads + hq) * kPartStride;
-        if (qd == 0) *reinterpret_cast<float4*>(dst) = make_float4(sHd[SL + h], sHd[2 * SL + h], 0.f, 0.f);
+        if (qd == 0) *reinterpret_cast<float4*>(dst) = make_float4(Mt, Lt, 0.f, 0.f);
         *reinterpret_cast<float4*>(dst + 4 + 4 * qd) = O;
       } else if (a.out_f32) {
         *reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow) =
@@ -661,20 +676,25 @@ __global__ void __launch_bounds__(Shape<NSET>::threads, 1) k_decode(const __grid
   // it overlaps that kernel. The lengths and the cache are read after the wait.
   int t1 = t0;
   if (t0 < a.max_len) {
-    // warm L2 with this block's packed rows (all of them lie below the capacity); the reads
-    // proper come after the dependency wait (L2 is the point of coherence for the append)
+    // L2 prefetch of each warp's first chunk (one bulk prefetch per plane by the TMA unit),
+    // which lands during the prologue; every later chunk's rows are loaded one chunk ahead.
+    // (Warming L2 with the block's whole token range instead kept the issuing warps busy
+    // for microseconds, and its lines were read long before their use.) Ranges start
+    // 16-byte aligned (aligned planes, a capacity that is a multiple of 16 rows, chunks of 32
+    // rows) and, rounded up to 16 bytes, end inside the plane. The reads proper come after
+    // the dependency wait (L2 is the point of coherence for the append).
     {
-      const int tp1 = min(a.max_len, t0 + a.tokens_per_split);
-      const int n = tp1 - t0;
-      const uint8_t* rng[5] = {a.k_idx + (kvrow + t0) * IB, a.k_sgn + (kvrow + t0) * 16,
-                               reinterpret_cast<const uint8_t*>(a.k_nrm) + (kvrow + t0) * Lo::NB,
-                               a.v_q + (kvrow + t0) * Lo::VQB,
-                               reinterpret_cast<const uint8_t*>(a.v_par) + (kvrow + t0) * 16};
-      const int len_b[5] = {n * IB, PROD ? n * 16 : 0, n * Lo::NB, n * Lo::VQB, VB ? n * 16 : 0};
-#pragma unroll
-      for (int r = 0; r < 5; ++r)
-        for (int off = threadIdx.x * 128; off < len_b[r]; off += NT * 128)
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(rng[r] + off));
+      const int cf = t0 + 32 * warp;
+      const int nf = min(32, min(a.max_len, t0 + a.tokens_per_split) - cf);
+      if (nf > 0 && lane < 5) {
+        const uint8_t* base[5] = {a.k_idx + (kvrow + cf) * IB, a.k_sgn + (kvrow + cf) * 16,
+                                  reinterpret_cast<const uint8_t*>(a.k_nrm) + (kvrow + cf) * Lo::NB,
+                                  a.v_q + (kvrow + cf) * Lo::VQB,
+                                  reinterpret_cast<const uint8_t*>(a.v_par) + (kvrow + cf) * 16};
+        const int len[5] = {nf * IB, PROD ? nf * 16 : 0, nf * Lo::NB, nf * Lo::VQB, VB ? nf * 16 : 0};
+        const int len16 = (len[lane] + 15) & ~15;
+        if (len16 > 0) bulk_prefetch_l2(base[lane], static_cast<uint32_t>(len16));
+      }
     }
 
     // ---------------- prologue: rotate q, project with S_rot, build the tables
