@@ -107,6 +107,10 @@ __host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / 
 // bytes form two lookup segments: I (index bytes; grouped: the outlier group) and S (prod:
 // the QJL sign bytes; grouped: the normal group, padded with zero bytes to whole 8-byte
 // blocks). Each segment accumulates its own sum; the two norms scale them.
+// A warp's per-head record after the main loop (floats): m at 0, the lanes' sums from
+// kWRecL, their largest logits from kWRecX, the two half-warps' outputs from kWRecO.
+constexpr int kWRecL = 4, kWRecX = kWRecL + 32, kWRecO = kWRecX + 32, kWRec = kWRecO + 2 * kD;
+
 template <int MB, int VB, int K, int NSET, int NH>
 struct Lay {
   static constexpr int SL = Shape<NSET>::slots, NW = Shape<NSET>::warps;
@@ -149,10 +153,10 @@ struct Lay {
   static constexpr int qlo = qhi + 8 * kQStride;
   static constexpr int qinv = qlo + 8 * kQStride;
   static constexpr int pro_end = qinv + 32;
-  // after the main loop, from byte 0: the warps' partials [NW][SL][kPartStride] f32, or the
-  // last block's merge of split maxima, sums and weights, and per-slice partial sums
-  static constexpr int merge = NW * SL * kPartStride * 4;
-  static constexpr int last = 3 * SL * 256 * 4 + 4 * SL * 4 + NW * 32 * 16;
+  // after the main loop, from byte 0: the warps' records [NW][SL][kWRec] f32, or the
+  // last block's slice maxima and sums and slice partial outputs
+  static constexpr int merge = NW * SL * kWRec * 4;
+  static constexpr int last = 16 * 8 * SL + NW * SL * 32 * 16;
   static constexpr int total0 = warps_end > pro_end ? warps_end : pro_end;
   static constexpr int total1 = total0 > merge ? total0 : merge;
   static constexpr int total = total1 > last ? total1 : last;
@@ -164,11 +168,6 @@ struct Lay {
 // their memory is visible (a no-op when the kernel was launched without the attribute).
 __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
-}
-
-// L2 prefetch of [p, p + bytes) by the TMA unit (p 16-byte aligned, bytes a multiple of 16)
-__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -473,11 +472,17 @@ __device__ __forceinline__ void decode_prologue(const DecodeArgs& a, uint8_t* sm
   __syncthreads();
 }
 
-// The block's partial from its NREC records [NREC][SL][kPartStride] at smem (m: the record's
-// reference maximum, l: the sum relative to it, max: its largest logit, o[128] from float 4):
+// The block's partial from its warps' NREC records [NREC][SL][kWRec] at smem (m: the warp's
+// reference maximum; per lane: its sum relative to m and its largest logit; the outputs of
+// the two half-warps, 128 channels each):
 // relative to the block's largest logit M, written as the output (one split), as a
 // context-parallel record, or as a split partial; the last block of a (sequence, head group)
 // to finish then merges every split. Every thread of the block calls this.
+// Last-block merge scratch: slice (M, L) pairs at 0, slice outputs from kMergeAccOff (at most
+// 16 slices).
+template <int SL>
+__host__ __device__ constexpr int kMergeAccOff() { return 16 * 8 * SL; }
+
 template <int NH, int SL, int NT, int NREC>
 __device__ __forceinline__ void decode_merge(const DecodeArgs& a, uint8_t* smem, int* sLastp,
                                              const int16_t* gheads, int nh, int b, int split) {
@@ -486,26 +491,29 @@ __device__ __forceinline__ void decode_merge(const DecodeArgs& a, uint8_t* smem,
   float* sM = reinterpret_cast<float*>(smem);
   __syncthreads();
   if (warp < nh) {
-    // partial of this block relative to its largest logit M
+    // partial of this block relative to its largest logit M, from the warps' records (lane:
+    // channels 4 lane .. 4 lane + 3); an empty record (m = -inf, l = 0, o = 0) gets weight 0
     const int h = warp, hq = gheads[h];
-    float M = -INFINITY;
+    float mloc = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NREC; ++w) M = fmaxf(M, sM[(w * SL + h) * kPartStride + 2]);
-    float Lsum = 0.f, O[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int w = 0; w < NREC; ++w) mloc = fmaxf(mloc, sM[(w * SL + h) * kWRec + kWRecX + lane]);
+    const float M = warp_max(mloc);
+    float Lp = 0.f, O[4] = {0.f, 0.f, 0.f, 0.f};
     if (M != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < NREC; ++w) {
-        const float* src = sM + (w * SL + h) * kPartStride;
-        if (src[0] == -INFINITY) continue;
+        const float* src = sM + (w * SL + h) * kWRec;
         const float f = ex2(src[0] - M);
-        Lsum = fmaf(f, src[1], Lsum);
-        const float4 ov = *reinterpret_cast<const float4*>(src + 4 + 4 * lane);
-        O[0] = fmaf(f, ov.x, O[0]);
-        O[1] = fmaf(f, ov.y, O[1]);
-        O[2] = fmaf(f, ov.z, O[2]);
-        O[3] = fmaf(f, ov.w, O[3]);
+        Lp = fmaf(f, src[kWRecL + lane], Lp);
+        const float4 o0 = *reinterpret_cast<const float4*>(src + kWRecO + 4 * lane);
+        const float4 o1 = *reinterpret_cast<const float4*>(src + kWRecO + kD + 4 * lane);
+        O[0] = fmaf(f, o0.x + o1.x, O[0]);
+        O[1] = fmaf(f, o0.y + o1.y, O[1]);
+        O[2] = fmaf(f, o0.z + o1.z, O[2]);
+        O[3] = fmaf(f, o0.w + o1.w, O[3]);
       }
     }
+    const float Lsum = warp_sum(Lp);
     const int64_t orow = (static_cast<int64_t>(b) * a.n_q_heads + hq) * kD + 4 * lane;
     if (a.n_splits == 1 && a.part_out != nullptr) {
       float* dst = a.part_out + (static_cast<int64_t>(b) * a.n_q_heads + hq) * kPartStride;
@@ -547,13 +555,13 @@ __device__ __forceinline__ void decode_merge(const DecodeArgs& a, uint8_t* smem,
   __syncthreads();
   if (!sLast) return;
   // Item (head, channel quad, split slice) loads the (maximum, sum, output quad) records of
-  // its splits in one round trip (batches of 8) and merges them relative to their largest
-  // maximum; the slices are then merged in shared memory.
+  // its splits in batches of 16 (one round trip each; one batch in practice) and merges them
+  // relative to their largest maximum; the slices are then merged in shared memory.
   {
     const int S = a.n_splits;
     const int G = NT / (32 * nh);  // split slices
-    float2* sML = reinterpret_cast<float2*>(smem);                  // [slice][head] (M, L)
-    float4* sAcc = reinterpret_cast<float4*>(smem + 16 * 8 * SL);   // [slice][head][32]
+    float2* sML = reinterpret_cast<float2*>(smem);                        // [slice][head] (M, L)
+    float4* sAcc = reinterpret_cast<float4*>(smem + kMergeAccOff<SL>());  // [slice][head][32]
     const float* base = a.part + static_cast<int64_t>(b) * a.n_q_heads * S * kPartStride;
     if (threadIdx.x < G * 32 * nh) {
       const int h = threadIdx.x / (32 * G), r = threadIdx.x - h * 32 * G;
@@ -561,11 +569,12 @@ __device__ __forceinline__ void decode_merge(const DecodeArgs& a, uint8_t* smem,
       const float* src = base + static_cast<int64_t>(gheads[h]) * S * kPartStride;
       float M = -INFINITY, L = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int sp0 = g; sp0 < S; sp0 += 8 * G) {
-        float2 ml[8];
-        float4 v[8];
+      constexpr int U = 16;
+      for (int sp0 = g; sp0 < S; sp0 += U * G) {
+        float2 ml[U];
+        float4 v[U];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < U; ++u) {
           const int sp = sp0 + u * G;
           if (sp < S) {
             const float* rec = src + static_cast<int64_t>(sp) * kPartStride;
@@ -578,14 +587,14 @@ __device__ __forceinline__ void decode_merge(const DecodeArgs& a, uint8_t* smem,
         }
         float mb = M;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) mb = fmaxf(mb, ml[u].x);
+        for (int u = 0; u < U; ++u) mb = fmaxf(mb, ml[u].x);
         if (mb == -INFINITY) continue;  // no token so far
         const float al = ex2(M - mb);   // 0 while M = -inf
         L *= al;
         acc.x *= al; acc.y *= al; acc.z *= al; acc.w *= al;
         M = mb;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < U; ++u) {
           const float f = ex2(ml[u].x - M);  // 0 for an empty split (m = -inf)
           L = fmaf(f, ml[u].y, L);
           acc.x = fmaf(f, v[u].x, acc.x); acc.y = fmaf(f, v[u].y, acc.y);
@@ -676,24 +685,25 @@ __global__ void __launch_bounds__(Shape<NSET>::threads, 1) k_decode(const __grid
   // it overlaps that kernel. The lengths and the cache are read after the wait.
   int t1 = t0;
   if (t0 < a.max_len) {
-    // L2 prefetch of each warp's first chunk (one bulk prefetch per plane by the TMA unit),
-    // which lands during the prologue; every later chunk's rows are loaded one chunk ahead.
-    // (Warming L2 with the block's whole token range instead kept the issuing warps busy
-    // for microseconds, and its lines were read long before their use.) Ranges start
-    // 16-byte aligned (aligned planes, a capacity that is a multiple of 16 rows, chunks of 32
-    // rows) and, rounded up to 16 bytes, end inside the plane. The reads proper come after
-    // the dependency wait (L2 is the point of coherence for the append).
+    // L2 prefetch of each warp's first chunk (its lanes spread the 128-byte lines of the five
+    // planes), which lands during the prologue; every later chunk's rows are loaded one chunk
+    // ahead. (Warming L2 with the block's whole token range instead kept the issuing warps
+    // busy for microseconds, and its lines were read long before their use.) The rows lie
+    // below the capacity; the reads proper come after the dependency wait (L2 is the point of
+    // coherence for the append).
     {
       const int cf = t0 + 32 * warp;
       const int nf = min(32, min(a.max_len, t0 + a.tokens_per_split) - cf);
-      if (nf > 0 && lane < 5) {
+      if (nf > 0) {
         const uint8_t* base[5] = {a.k_idx + (kvrow + cf) * IB, a.k_sgn + (kvrow + cf) * 16,
                                   reinterpret_cast<const uint8_t*>(a.k_nrm) + (kvrow + cf) * Lo::NB,
                                   a.v_q + (kvrow + cf) * Lo::VQB,
                                   reinterpret_cast<const uint8_t*>(a.v_par) + (kvrow + cf) * 16};
         const int len[5] = {nf * IB, PROD ? nf * 16 : 0, nf * Lo::NB, nf * Lo::VQB, VB ? nf * 16 : 0};
-        const int len16 = (len[lane] + 15) & ~15;
-        if (len16 > 0) bulk_prefetch_l2(base[lane], static_cast<uint32_t>(len16));
+#pragma unroll
+        for (int r = 0; r < 5; ++r)
+          for (int off = 128 * lane; off < len[r]; off += 32 * 128)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(base[r] + off));
       }
     }
 
@@ -920,24 +930,23 @@ __global__ void __launch_bounds__(Shape<NSET>::threads, 1) k_decode(const __grid
 
   // ---------------- merge the warps of this block
   __syncthreads();
-  float* sM = reinterpret_cast<float*>(smem);  // [warp][head][kPartStride]: m, l, max, o
+  // Each warp's record per head: its reference maximum m, the lanes' sums and largest
+  // logits, and the outputs of both half-warps (disjoint tokens of the same channels); the
+  // block merge reduces them across lanes once per head instead of once per warp and head.
+  float* sM = reinterpret_cast<float*>(smem);  // [warp][head][kWRec]
+  {
+    const int hw = lane >> 4, j16 = lane & 15;
 #pragma unroll
-  for (int h = 0; h < NH; ++h) {
-    // the two half-warps hold disjoint tokens of the same channels
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 v = up2(o[h][k]);
-      o[h][k] = add2(o[h][k], pk2(__shfl_xor_sync(kFull, v.x, 16), __shfl_xor_sync(kFull, v.y, 16)));
-    }
-    const float lt = warp_sum(l[h]);
-    const float mt = warp_max(mx[h]);
-    if (h < nh) {
-      float* dst = sM + (warp * SL + h) * kPartStride;
-      if (lane == 0) { dst[0] = m[h]; dst[1] = lt; dst[2] = mt; }
-      if (lane < 16) {
+    for (int h = 0; h < NH; ++h) {
+      if (h < nh) {
+        float* dst = sM + (warp * SL + h) * kWRec;
+        if (lane == 0) dst[0] = m[h];
+        dst[kWRecL + lane] = l[h];
+        dst[kWRecX + lane] = mx[h];
         const float2 v0 = up2(o[h][0]), v1 = up2(o[h][1]), v2 = up2(o[h][2]), v3 = up2(o[h][3]);
-        *reinterpret_cast<float4*>(dst + 4 + 8 * lane) = make_float4(v0.x, v0.y, v1.x, v1.y);
-        *reinterpret_cast<float4*>(dst + 8 + 8 * lane) = make_float4(v2.x, v2.y, v3.x, v3.y);
+        float* od = dst + kWRecO + kD * hw + 8 * j16;
+        *reinterpret_cast<float4*>(od) = make_float4(v0.x, v0.y, v1.x, v1.y);
+        *reinterpret_cast<float4*>(od + 4) = make_float4(v2.x, v2.y, v3.x, v3.y);
       }
     }
   }
