@@ -990,13 +990,16 @@ constexpr bool two_sets_fit() {
   else return Lay<MB, VB, K, 2, 8>::fits;
 }
 
-// Heads per block template: one set 2 or 4, two sets 6 or 8.
+// Heads per block template: one set 2 or 4, two sets 6, 7 or 8 (each P.V step works on
+// every head slot of the template, so the 7-head groups of 7:1 grouped-query attention skip
+// the eighth).
 template <int MB, int VB, int K>
 tq_status run_decode_shape(const DecodeArgs& a, dim3 grid, int max_heads, bool two, bool pdl,
                            cudaStream_t st) {
   if constexpr (two_sets_fit<MB, VB, K>()) {
     if (two) {
       if (max_heads <= 6) return run_decode<MB, VB, 6, K, 2>(a, grid, pdl, st);
+      if (max_heads == 7) return run_decode<MB, VB, 7, K, 2>(a, grid, pdl, st);
       return run_decode<MB, VB, 8, K, 2>(a, grid, pdl, st);
     }
   }
