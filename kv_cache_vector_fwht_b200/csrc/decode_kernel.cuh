@@ -990,9 +990,8 @@ constexpr bool two_sets_fit() {
   else return Lay<MB, VB, K, 2, 8>::fits;
 }
 
-// Heads per block template: one set 2 or 4, two sets 6, 7 or 8 (each P.V step works on
-// every head slot of the template, so the 7-head groups of 7:1 grouped-query attention skip
-// the eighth).
+// Heads per block template: one set 2, 3 or 4, two sets 6, 7 or 8 (each P.V step works on
+// every head slot of the template, so groups of 3 or 7 heads skip the empty slot).
 template <int MB, int VB, int K>
 tq_status run_decode_shape(const DecodeArgs& a, dim3 grid, int max_heads, bool two, bool pdl,
                            cudaStream_t st) {
@@ -1004,6 +1003,7 @@ tq_status run_decode_shape(const DecodeArgs& a, dim3 grid, int max_heads, bool t
     }
   }
   if (max_heads <= 2) return run_decode<MB, VB, 2, K, 1>(a, grid, pdl, st);
+  if (max_heads == 3) return run_decode<MB, VB, 3, K, 1>(a, grid, pdl, st);
   return run_decode<MB, VB, 4, K, 1>(a, grid, pdl, st);
 }
 
