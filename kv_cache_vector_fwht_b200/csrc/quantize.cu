@@ -15,6 +15,7 @@
 // (h = 1): the first butterfly stage of H_128 = [[H_64, H_64], [H_64, -H_64]]. The remaining
 // six stages run in registers, so lane h ends with coordinates [64h, 64h + 64) of y.
 #include <cfloat>
+#include <cstddef>
 
 #include "tq_device.cuh"
 #include "tq_internal.h"
@@ -70,7 +71,25 @@ __global__ void __launch_bounds__(256) k_keys_full(KeyArgs a) {
   for (int k = 0; k < 4; ++k) sb[k] = tab->sign_bits[k];
 
   if constexpr (PROD) {
-    for (int e = threadIdx.x; e < kD * kD; e += blockDim.x) sST[e] = __half2float(tab->s_rot_t[e]);
+    // 16-byte loads of 8 fp16 entries each (a small batch runs 2-warp blocks, for which
+    // element-wise loads made this staging most of the kernel's time)
+    static_assert(offsetof(DevTables, s_rot_t) % 16 == 0, "16-byte aligned S_rot^T");
+    const uint4* src = reinterpret_cast<const uint4*>(tab->s_rot_t);
+#pragma unroll 4
+    for (int e8 = threadIdx.x; e8 < kD * kD / 8; e8 += blockDim.x) {
+      const uint4 v = __ldg(src + e8);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      float f[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 p = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+        f[2 * i] = p.x;
+        f[2 * i + 1] = p.y;
+      }
+      float4* d = reinterpret_cast<float4*>(sST + 8 * e8);
+      d[0] = make_float4(f[0], f[1], f[2], f[3]);
+      d[1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
     __syncthreads();
   }
 
