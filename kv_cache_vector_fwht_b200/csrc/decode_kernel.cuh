@@ -132,11 +132,11 @@ struct Lay {
   static constexpr int lutI = 0;
   static constexpr int lutS = lutI + NSET * SETI;
   static constexpr int tables = lutS + NSET * SETS;
-  // per-warp slot: (p, p, p', p') float4 pairs [NH2][32], value parameters [4][kVpStride],
+  // per-warp slot: softmax weights p of 4 heads a float4 [NH4][32], value parameters [4][kVpStride],
   // value codes [32][VQB]
-  static constexpr int NH2 = (NH + 1) / 2;
+  static constexpr int NH4 = (NH + 3) / 4;
   static constexpr int oPP = 0;
-  static constexpr int oVP = oPP + NH2 * 32 * 16;
+  static constexpr int oVP = oPP + NH4 * 32 * 16;
   static constexpr int wv = round_up(tables, 128);
   static constexpr int budget = 227 * 1024 - 512;                  // leave room for static smem
   // value parameters as float4 (16 s16-scaled pairs and offsets) where the slots fit, else
@@ -650,7 +650,7 @@ __global__ void __launch_bounds__(Shape<NSET>::threads, 1) k_decode(const __grid
   constexpr int CS = Shape<NSET>::chunk_stride;
   constexpr int SL = Shape<NSET>::slots;
   constexpr bool PROD = K == kProd, GRP = K == kGrp, TWO = K != kMse;
-  constexpr int IB = Lo::IB, PI = Lo::PI, KW = Lo::KW, NH2 = Lo::NH2;
+  constexpr int IB = Lo::IB, PI = Lo::PI, KW = Lo::KW, NH4 = Lo::NH4;
   static_assert(NH >= 1 && NH <= SL, "heads per block");
   static_assert(Lo::fits, "decode shared memory budget");
   constexpr bool HAS_V = VB != 0;
@@ -714,7 +714,7 @@ __global__ void __launch_bounds__(Shape<NSET>::threads, 1) k_decode(const __grid
 
     // ---------------- main loop over this warp's chunks
     uint8_t* wslot = smem + Lo::wv + warp * Lo::WB;
-    float4* sPP = reinterpret_cast<float4*>(wslot + Lo::oPP);     // [NH2][32]
+    float4* sP4 = reinterpret_cast<float4*>(wslot + Lo::oPP);     // [NH4][32] p of 4 heads
     uint8_t* sVP = wslot + Lo::oVP;                               // [4][kVpStride] params
     uint8_t* sVQ = wslot + Lo::oVQ;                               // [32][VQB]
     const uint8_t* vq_rows = a.v_q + kvrow * Lo::VQB;
@@ -854,9 +854,11 @@ __global__ void __launch_bounds__(Shape<NSET>::threads, 1) k_decode(const __grid
           mx[h] = fmaxf(mx[h], valid ? sc[h] : -INFINITY);
         }
 #pragma unroll
-        for (int k = 0; k < NH2; ++k) {
-          const float pa = p[2 * k], pb = 2 * k + 1 < NH ? p[(2 * k + 1) % NH] : 0.f;
-          sPP[k * 32 + lane] = make_float4(pa, pa, pb, pb);
+        for (int k = 0; k < NH4; ++k) {
+          float q4[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) q4[i] = 4 * k + i < NH ? p[(4 * k + i) % NH] : 0.f;
+          sP4[k * 32 + lane] = make_float4(q4[0], q4[1], q4[2], q4[3]);
         }
         {
           // this token's group parameters (zeros past the range: v = 0 there)
@@ -907,14 +909,19 @@ __global__ void __launch_bounds__(Shape<NSET>::threads, 1) k_decode(const __grid
                               __uint_as_float(0x3f800000u | (w & 0x00780000u))), SP, CP);
             }
           }
+          // p of 4 heads per 16-byte load; the (p, p) pairs are formed in registers
 #pragma unroll
-          for (int k2 = 0; k2 < NH2; ++k2) {
-            const float4 pp = sPP[k2 * 32 + tok];
-            const uint64_t pa = pk2(pp.x, pp.y), pb = pk2(pp.z, pp.w);
+          for (int k4 = 0; k4 < NH4; ++k4) {
+            const float4 pp = sP4[k4 * 32 + tok];
+            const float pv[4] = {pp.x, pp.y, pp.z, pp.w};
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              o[2 * k2][k] = fma2(pa, v[k], o[2 * k2][k]);
-              if (2 * k2 + 1 < NH) o[(2 * k2 + 1) % NH][k] = fma2(pb, v[k], o[(2 * k2 + 1) % NH][k]);
+            for (int i = 0; i < 4; ++i) {
+              const int h = 4 * k4 + i;
+              if (h < NH) {
+                const uint64_t ph = pk2(pv[i], pv[i]);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) o[h][k] = fma2(ph, v[k], o[h][k]);
+              }
             }
           }
         }
