@@ -27,6 +27,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import subprocess
 import sys
 import time
@@ -114,12 +115,22 @@ def load_peaks():
         return 6650.0, "fallback"
 
 
+def _code_only(text: str) -> str:
+    """C/CUDA source without its comments and trailing blanks: what the compiler sees, so that
+    editing a comment does not orphan the traffic recorded for the code. (The kernel sources
+    put no comment markers inside string literals.)"""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def source_sha(files) -> str:
-    """Short hash of kernel sources (the key under which ncu DRAM traffic was recorded)."""
+    """Short hash of the kernel sources' code (the key under which ncu DRAM traffic was
+    recorded)."""
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "kv_cache_vector_fwht_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "kv_cache_vector_fwht_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

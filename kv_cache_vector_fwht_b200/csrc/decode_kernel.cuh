@@ -32,7 +32,8 @@
 //            half-warps take alternate tokens, lane j of a half owns channels 8j .. 8j + 7,
 //            dequantizes them once (v = (1 + code/16) * 16 s16 + (mn16 - 16 s16), exact
 //            field insertion and one packed FMA per channel pair) and accumulates every head
-//            in packed fp32x2 FMAs with the head's (p, p) pair read as a shared broadcast.
+//            in packed fp32x2 FMAs; the token's p of 4 heads is one shared 16-byte
+//            broadcast and each head's (p, p) operand pair is formed in registers.
 // Each block merges its warps and writes a partial (m, l, o) with m the largest logit; the
 // last block of a (sequence, head group) to finish merges all partials (an atomic counter,
 // no waiting), or writes the merged partial itself for a context-parallel decode.
@@ -236,12 +237,18 @@ template <int ROWB, int NS, int SETB>
 __device__ __forceinline__ void block_lookups3(uint64_t (&acc)[NS][2], uint32_t R0, uint32_t R1,
                                                const uint8_t* tab, int blk,
                                                const uint32_t (&rot16)[8]) {
+  const uint32_t S0 = R0 << 1, S1 = R1 << 1;  // bit 7 of every byte is clear: no carries
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const uint32_t R = i < 4 ? R0 : R1;
-    const uint32_t v = (R >> (8 * (i & 3))) & 0xffu;
-    const int msk = static_cast<int>(v << 25) >> 31;
-    const uint32_t e = v ^ (static_cast<uint32_t>(msk) & 0x77u);
+    const uint32_t R2 = i < 4 ? S0 : S1;
+    // byte i zero-extended, and the mirror flag (bit 6, moved to bit 7 in R << 1) replicated
+    // over a word: one byte permute each
+    uint32_t v, ms;
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(v) : "r"(R), "r"(static_cast<uint32_t>((i & 3) | 0x4440)));
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(ms) : "r"(R2), "r"(static_cast<uint32_t>((8 | (i & 3)) * 0x1111)));
+    const int msk = static_cast<int>(ms);
+    const uint32_t e = v ^ (ms & 0x77u);
     lut_acc<NS, SETB>(acc, tab + 128 * blk + e * ROWB + rot16[i], sign_pair(msk));
   }
 }
