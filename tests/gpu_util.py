@@ -75,3 +75,24 @@ def upload_cache(cache, oc: dict) -> None:
         put(cache.v_q, oc["v_q"])
         put(cache.v_params, oc["v_params"])
     cache.set_lengths(oc["len"])
+
+
+def download_pair(cache, b: int, h: int, n: int) -> dict:
+    """The first n rows of (sequence b, KV head h) of a KVCache as an oracle cache dict with
+    one sequence and one KV head (the reverse of upload_cache for one pair)."""
+    rows = cache.rows(b, h)
+    lay_shape = {"k_norms": None, "v_params": (4, 2)}
+    out = {}
+    for name in ("k_idx", "k_norms", "k_signs", "v_q", "v_params"):
+        t = getattr(cache, name, None)
+        if t is None:
+            out[name] = None
+            continue
+        a = t[rows][:n].cpu().numpy()
+        if a.dtype == np.int16:
+            a = a.view(np.uint16)
+        shape = lay_shape.get(name)
+        a = a.reshape((n,) + shape) if shape else a.reshape(n, -1)
+        out[name] = a[None, None]
+    out["len"] = np.array([n], dtype=np.int64)
+    return out

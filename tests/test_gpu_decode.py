@@ -10,7 +10,7 @@ import torch
 
 import oracle as O
 import workloads as W
-from gpu_util import oracle_cache, require_cuda, to_device, to_np_planes, upload_cache
+from gpu_util import download_pair, oracle_cache, require_cuda, to_device, to_np_planes, upload_cache
 from parity import check_attention, check_key_parity, check_scores
 
 pytestmark = pytest.mark.gpu
@@ -223,16 +223,54 @@ def test_decode_full_config_decode_s():
 
 
 def test_decode_full_config_decode_l():
-    """Batch 8, 28/4 GQA, context 32768 with planted keys; sampled (sequence, KV head)
-    pairs; the planted keys dominate attention for the first head of each group."""
+    """Batch 8, 28/4 GQA, context 32768 with planted keys; sampled (sequence, KV head) pairs
+    quantized by the oracle, all 7 heads of each against the oracle's decode."""
     out = _full_decode(3, [(0, 0), (7, 3), (3, 1)], torch.bfloat16)
     assert np.all(np.isfinite(out))
+
+
+def test_decode_l_every_pair_and_planted_scores():
+    """decode-l at full size on the GPU-quantized cache (batch 8, 28/4 GQA, 32768 tokens with
+    16 planted keys 0.9 q + 0.1 noise per pair): every (sequence, KV head) pair's 7 heads
+    against the oracle's decode of the same packed rows (bf16 output), and the scores of the
+    planted keys for the query head they were planted for against the oracle's scores. With
+    row scales up to 20 the planted keys do not dominate attention; their softmax mass is
+    printed."""
+    require_cuda()
+    cfg = W.WORKLOADS[3]
+    B, Hq, Hkv, N = cfg["batch"], cfg["n_q_heads"], cfg["n_kv_heads"], cfg["ctx"]
+    K, V, Q, pos = W.decode_inputs(3, B, Hq, Hkv, N, planted=cfg["planted"])
+    qo = O.build_quantizer(128, cfg["key_bits"], "prod", cfg["qseed"])
+    qg = tq.tq_build_codebook(128, cfg["key_bits"], "prod", cfg["qseed"])
+    G, vb = Hq // Hkv, cfg["value_bits"]
+    cache = tq.KVCache(qg, B, Hkv, N, value_bits=vb, device="cuda:0")
+    tq.tq_append(qg, cache, to_device(K, torch.bfloat16), to_device(V, torch.bfloat16))
+    out, sc, _ = run_decode(qg, cache, Q, torch.bfloat16, torch.bfloat16, scores_ld=N)
+    worst = 0.0
+    for b in range(B):
+        for kv in range(Hkv):
+            oc = download_pair(cache, b, kv, N)
+            heads = list(range(kv * G, (kv + 1) * G))
+            ref, rs = O.decode_attention(qo, oc, Q[b:b + 1, heads].astype(np.float64),
+                                         head_map=np.zeros(G, dtype=int), value_bits=vb,
+                                         want_scores=True)
+            worst = max(worst, check_attention(out[b, heads], ref[0], True))
+            h = kv * G
+            p = pos[b, kv]
+            n16 = O.fp16_from_bits(oc["k_norms"][0, 0, :, 0])
+            check_scores(sc[b, h][p], rs[0][0][p], np.linalg.norm(Q[b, h]), n16[p])
+            s = rs[0][0] / np.sqrt(128.0)
+            w = np.exp(s - s.max())
+            if b == 0:
+                print("pair", b, kv, "planted softmax mass", float(w[p].sum() / w.sum()))
+    print("decode-l every pair: worst", worst)
 
 
 def test_decode_stream_steps():
     """Streaming decode: context 131072, 64/8 GQA, 4-bit prod keys, 4-bit values; each step
     appends one token per KV head on the GPU, then decodes. Appended rows are checked
-    against the oracle, and the decode after each step against the oracle's cache."""
+    against the oracle, the decode after each step against the oracle's cache (one KV head),
+    and after the last step every KV head against the oracle's decode of the GPU's rows."""
     require_cuda()
     cfg = W.WORKLOADS[5]
     B, Hq, Hkv, N = 1, cfg["n_q_heads"], cfg["n_kv_heads"], cfg["ctx"]
@@ -266,6 +304,15 @@ def test_decode_stream_steps():
         ref, _ = O.decode_attention(qo, step_oc, Q[:, heads].astype(np.float64),
                                     head_map=np.zeros(G, dtype=int), value_bits=4)
         check_attention(out[0, heads], ref[0], False)
+    # after the last step, every KV head's 8 query heads against the oracle's decode of the
+    # GPU's own packed rows (the appended token included)
+    n = N + steps
+    for kvh in range(Hkv):
+        oc_h = download_pair(cache, 0, kvh, n)
+        hs = list(range(kvh * G, (kvh + 1) * G))
+        ref, _ = O.decode_attention(qo, oc_h, Q[:, hs].astype(np.float64),
+                                    head_map=np.zeros(G, dtype=int), value_bits=4)
+        check_attention(out[0, hs], ref[0], False)
 
 
 def _slice_oracle_cache(oc, start, stop):
