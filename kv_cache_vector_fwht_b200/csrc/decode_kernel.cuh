@@ -562,7 +562,7 @@ __device__ __forceinline__ void decode_merge(const DecodeArgs& a, uint8_t* smem,
   __syncthreads();
   if (!sLast) return;
   // Item (head, channel quad, split slice) loads the (maximum, sum, output quad) records of
-  // its splits in batches of 16 (one round trip each; one batch in practice) and merges them
+  // its splits in batches of 16 (one round trip each) and merges them
   // relative to their largest maximum; the slices are then merged in shared memory.
   {
     const int S = a.n_splits;
