@@ -74,6 +74,19 @@ __device__ __forceinline__ uint32_t h2_bits(float lo, float hi) {
 }
 
 // 1.0f if a > b else 0.0f (an exact compare)
+// m + 1/2 with m = #{k < 7 : a > T[OFF + k]} for ascending T[OFF .. OFF + 6] (the positive
+// thresholds of a 16-level codebook), by binary search: the same strict compares as the
+// ladder over all seven, along one path of three, so the count is identical.
+template <int OFF, int N>
+__device__ __forceinline__ float mag_half7(float a, const float (&T)[N]) {
+  static_assert(OFF + 7 <= N, "seven thresholds");
+  const bool b4 = a > T[OFF + 3];
+  const bool b2 = a > (b4 ? T[OFF + 5] : T[OFF + 1]);
+  const float t1 = b4 ? (b2 ? T[OFF + 6] : T[OFF + 4]) : (b2 ? T[OFF + 2] : T[OFF + 0]);
+  const bool b1 = a > t1;
+  return (b4 ? 4.f : 0.f) + (b2 ? 2.f : 0.f) + (b1 ? 1.5f : 0.5f);
+}
+
 __device__ __forceinline__ float gt_one(float a, float b) {
   float d;
   asm("set.gt.f32.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
@@ -326,13 +339,19 @@ __global__ void __launch_bounds__(128, 2)
             const float y0 = __uint_as_float(yv[2 * i]), y1 = __uint_as_float(yv[2 * i + 1]);
             const uint64_t s2 = pk2(gt_one(y0, 0.f), gt_one(y1, 0.f));
             const uint64_t sk2 = fma2(s2, pk2(2.f * kw, 2.f * kw), pk2(-kw, -kw));  // sigma kw
-            uint64_t w = fma2(sk2, pk2(0.5f, 0.5f), pi < GP / 2 ? wa : wb);
+            uint64_t w = pi < GP / 2 ? wa : wb;
             const float a0 = fabsf(y0), a1 = fabsf(y1);
+            if constexpr (H == 7 && !PROD) {
+              // 16 levels: m + 1/2 by binary search over the positive thresholds
+              w = fma2(sk2, pk2(mag_half7<0>(a0, TP), mag_half7<0>(a1, TP)), w);
+            } else {
+              w = fma2(sk2, pk2(0.5f, 0.5f), w);
 #pragma unroll
-            for (int t = 0; t < H; ++t) {
-              const uint64_t ind = pk2(gt_one(a0, TP[t]), gt_one(a1, TP[t]));
-              if constexpr (PROD) c2 = fma2(ind, dcsP2[t], c2);
-              w = fma2(ind, sk2, w);
+              for (int t = 0; t < H; ++t) {
+                const uint64_t ind = pk2(gt_one(a0, TP[t]), gt_one(a1, TP[t]));
+                if constexpr (PROD) c2 = fma2(ind, dcsP2[t], c2);
+                w = fma2(ind, sk2, w);
+              }
             }
             if (pi < GP / 2) wa = w;
             else wb = w;
@@ -526,10 +545,15 @@ __device__ __forceinline__ void decide16(const uint32_t (&yv)[16], const float (
     if constexpr (SYM) {
       const uint64_t s2 = pk2(gt_one(y0, 0.f), gt_one(y1, 0.f));
       const uint64_t sk2 = fma2(s2, pk2(2.f * wx, 2.f * wx), pk2(-wx, -wx));  // sigma kw
-      A = fma2(sk2, pk2(0.5f, 0.5f), A);
       const float a0 = fabsf(y0), a1 = fabsf(y1);
+      if constexpr (H == 7) {
+        // 16 levels: m + 1/2 by binary search over the positive thresholds
+        A = fma2(sk2, pk2(mag_half7<H + 1>(a0, T), mag_half7<H + 1>(a1, T)), A);
+      } else {
+        A = fma2(sk2, pk2(0.5f, 0.5f), A);
 #pragma unroll
-      for (int t = 0; t < H; ++t) A = fma2(pk2(gt_one(a0, T[H + 1 + t]), gt_one(a1, T[H + 1 + t])), sk2, A);
+        for (int t = 0; t < H; ++t) A = fma2(pk2(gt_one(a0, T[H + 1 + t]), gt_one(a1, T[H + 1 + t])), sk2, A);
+      }
     } else {
 #pragma unroll
       for (int t = 0; t < NT; ++t) A = fma2(pk2(gt_one(y0, T[t]), gt_one(y1, T[t])), kw, A);
