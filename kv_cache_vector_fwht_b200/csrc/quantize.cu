@@ -180,21 +180,28 @@ __global__ void __launch_bounds__(256) k_keys_full(KeyArgs a) {
 #pragma unroll
       for (int j = 0; j < 64; ++j) my[hf * 64 + j] = u[j];
       __syncwarp();
-      float acc[64];
+      // packed fp32x2 multiply-adds: the same rounding per element as scalar ones
+      uint64_t acc2[32];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) acc[j] = 0.f;
+      for (int j = 0; j < 32; ++j) acc2[j] = 0ull;
 #pragma unroll 2
       for (int i = 0; i < kD; ++i) {
         const float ri = my[i];
-        const float4* srow = reinterpret_cast<const float4*>(sST + i * kD + hf * 64);
+        const uint64_t ri2 = pk2(ri, ri);
+        const ulonglong2* srow = reinterpret_cast<const ulonglong2*>(sST + i * kD + hf * 64);
 #pragma unroll
         for (int q4 = 0; q4 < 16; ++q4) {
-          const float4 s = srow[q4];
-          acc[4 * q4 + 0] = fmaf(s.x, ri, acc[4 * q4 + 0]);
-          acc[4 * q4 + 1] = fmaf(s.y, ri, acc[4 * q4 + 1]);
-          acc[4 * q4 + 2] = fmaf(s.z, ri, acc[4 * q4 + 2]);
-          acc[4 * q4 + 3] = fmaf(s.w, ri, acc[4 * q4 + 3]);
+          const ulonglong2 sv = srow[q4];
+          acc2[2 * q4] = fma2(sv.x, ri2, acc2[2 * q4]);
+          acc2[2 * q4 + 1] = fma2(sv.y, ri2, acc2[2 * q4 + 1]);
         }
+      }
+      float acc[64];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float2 v = up2(acc2[j]);
+        acc[2 * j] = v.x;
+        acc[2 * j + 1] = v.y;
       }
       uint32_t sg0 = 0u, sg1 = 0u;
 #pragma unroll
